@@ -1,0 +1,379 @@
+/*
+ * moe_oracle.c -- CPU oracle for the gpt-oss-style MXFP4 expert-FFN MoE layer.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the package's
+ * smoke check and the CPU-baseline leg of the benchmark may load this library.
+ * It shares no code, header, table or helper with the CUDA path; it is a plain,
+ * slow, obviously-correct restatement of what the layer computes, in double
+ * precision, one element at a time.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P2] MoE-Infinity PR #152, "expert offloading Phase 2 -- MXFP4 dequant-on-copy
+ *        execution", section "Changes": mxfp4_dequantize golden test at rel-err 0.0;
+ *        the native forward keeps the scales, bias, [N, K//2] packed layout, gate/up
+ *        split, clamped SwiGLU and fp32 accumulation of the resident path.
+ *   [P3] FreeToken PR #838, "feat(gguf): serve gpt-oss gguf checkpoints on gpt_oss":
+ *        review item "NVFP4 down scale vs. down bias" (the result is sum w*(s*y + b),
+ *        never sum w*s*(y + b)); review item "w2_bias with
+ *        apply_router_weight_on_input" (with the router weight on the input both
+ *        expert biases must be absent); section "What it does" (swiglu alpha 1.702
+ *        and limit 7 are family constants; gate_up_bias [E, 2I] and down_bias [E, H];
+ *        gate/up bias added before the gated activation, down bias before the
+ *        routing weight; swigluoai is the uninterleaved spelling of the same math).
+ *   [P5] onnxruntime/mobius PR #719, "Add native GPT-OSS MXFP4 QMoE export",
+ *        sections "Summary" and "Validation": blocks [E, N, K/32, 16] (the same
+ *        bytes as [E, N, K/2]); E8M0 bytes 0x00..0xfe are valid, 0xff is rejected.
+ *   [P4] transformers PR #49431, "Restore GPT-OSS's router-masked expert-parallel
+ *        plan": the MXFP4 experts consume routing data (ids and weights), not a
+ *        dispatch of expert ids.
+ *   [MX] OCP Microscaling Formats (MX) v1.0: FP4 E2M1 element (1 sign, 2 exponent
+ *        bits with bias 1, 1 mantissa bit, no inf/NaN) and E8M0 scale (2^(b-127),
+ *        0xff = NaN).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   R1  element kk of a packed row lives in byte kk/2; the LOW nibble holds the
+ *       even element, the HIGH nibble the odd one.
+ *   R2  top-k takes the k largest logits in order (value descending, ties to the
+ *       lower expert index), then a softmax over those k values only.
+ *   R3  gate/up rows of the fused gate_up projection are interleaved:
+ *       gate = h[2i], up = h[2i+1].
+ *   R4  clamped SwiGLU: g = min(gate, limit), u = clamp(up, -limit, limit),
+ *       a = (u + 1) * g * sigmoid(alpha * g).
+ *   R5  a 0xff scale byte decodes to NaN (the pages reject it as invalid).
+ *
+ * Function that is not pinned by anything outside itself: none -- every entry
+ * point is checked against hand-written values, closed forms, invariants or a
+ * library routine by the CPU tests.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- planted mistakes (only the non-vacuity tests set these) ---------------- */
+enum {
+    ORACLE_DEFECT_NONE = 0,
+    ORACLE_DEFECT_NIBBLE_SWAP = 1,     /* high nibble taken as the even element      */
+    ORACLE_DEFECT_E8M0_BIAS_126 = 2,   /* 2^(b-126) instead of 2^(b-127)              */
+    ORACLE_DEFECT_GATE_ZERO = 3,       /* gate projection weights zeroed              */
+    ORACLE_DEFECT_NO_CLAMP = 4,        /* SwiGLU without the limit clamps             */
+    ORACLE_DEFECT_UNINTERLEAVED = 5,   /* gate = h[i], up = h[I + i]                  */
+    ORACLE_DEFECT_DOWN_BIAS_UNWEIGHTED = 6, /* sum (w*y + b) instead of sum w*(y + b) */
+    ORACLE_DEFECT_WOI_BIAS_WEIGHTED = 7,    /* router-weight-on-input: down bias scaled
+                                               by the routing weight                  */
+    ORACLE_DEFECT_DOWN_BIAS_IN_SCALE = 8,   /* down bias multiplied by the row's first
+                                               E8M0 block scale (scale after bias)    */
+};
+
+enum { ORACLE_FLAG_WEIGHT_ON_INPUT = 1 };
+
+/* ---- element formats [MX] ---------------------------------------------------- */
+
+/* E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+ * Exponent field 0 is subnormal: magnitude = m * 0.5. */
+double oracle_e2m1_value(int code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double mag;
+    if (e == 0)
+        mag = 0.5 * (double)m;
+    else
+        mag = ldexp(1.0 + 0.5 * (double)m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* E8M0: 2^(b - 127); 0xff is NaN (invalid per [P5] Validation; reading R5). */
+double oracle_e8m0_value(int b, int defect)
+{
+    if (b == 255)
+        return NAN;
+    return ldexp(1.0, b - (defect == ORACLE_DEFECT_E8M0_BIAS_126 ? 126 : 127));
+}
+
+/* double -> bfloat16 bits, round to nearest, ties to even, with subnormals
+ * and overflow to infinity.  bf16 keeps 8 significant bits; the spacing of
+ * representable values in [2^e, 2^(e+1)) is 2^(e-7), and below 2^-126 it is
+ * the fixed subnormal spacing 2^-133. */
+uint16_t oracle_double_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80);
+    int e2;
+    frexp(a, &e2);           /* a in [2^(e2-1), 2^e2) */
+    int e = e2 - 1;
+    if (e < -126)
+        e = -126;
+    double q = ldexp(1.0, e - 7);
+    double r = nearbyint(a / q) * q; /* default rounding mode: ties to even */
+    if (r >= ldexp(1.0, 128))
+        return (uint16_t)(sign | 0x7F80);
+    float f = (float)r;     /* exact: every bf16 value is a float */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+double oracle_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One weight element W[e, n, kk] of a packed bank: blocks [E, N, K/2],
+ * scales [E, N, K/32] ([P2] Changes: [N, K//2] layout; [P5] Summary: blocks
+ * [E, N, K/32, 16]).  Reading R1 for the nibble order. */
+static double weight_elem(const uint8_t *blocks, const uint8_t *scales,
+                          int64_t N, int64_t K, int64_t e, int64_t n, int64_t kk,
+                          int defect)
+{
+    int64_t row = e * N + n;
+    uint8_t byte = blocks[row * (K / 2) + kk / 2];
+    int even = (kk % 2) == 0;
+    if (defect == ORACLE_DEFECT_NIBBLE_SWAP)
+        even = !even;
+    int code = even ? (byte & 0xF) : (byte >> 4);
+    int s = scales[row * (K / 32) + kk / 32];
+    return oracle_e2m1_value(code) * oracle_e8m0_value(s, defect);
+}
+
+/* ---- standalone dequant-on-copy [P2] Changes ------------------------------- */
+/* out[e, n, kk] = bf16(E2M1(code) * 2^(s - 127)); every value with s <= 252 is
+ * exactly representable, so the golden test's rel-err 0.0 means bit-exact. */
+void oracle_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out,
+                       int64_t E, int64_t N, int64_t K, int defect)
+{
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t kk = 0; kk < K; ++kk)
+                out[(e * N + n) * K + kk] = oracle_double_to_bf16(
+                    weight_elem(blocks, scales, N, K, e, n, kk, defect));
+}
+
+/* ---- top-k routing (reading R2) --------------------------------------------- */
+/* ids[t, j] in selection order; weights[t, j] = exp(l_j - l_max) / sum over the
+ * k selected of exp(l_i - l_max), computed in double and stored as float. */
+void oracle_route(const float *logits, int64_t T, int64_t E, int k,
+                  int32_t *ids, float *weights)
+{
+    char *taken = (char *)malloc((size_t)E);
+    double *ex = (double *)malloc(sizeof(double) * (size_t)k);
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        memset(taken, 0, (size_t)E);
+        for (int j = 0; j < k; ++j) {
+            int64_t best = -1;
+            for (int64_t i = 0; i < E; ++i) {
+                if (taken[i])
+                    continue;
+                /* strictly greater keeps the lower index on ties */
+                if (best < 0 || l[i] > l[best])
+                    best = i;
+            }
+            taken[best] = 1;
+            ids[t * k + j] = (int32_t)best;
+        }
+        double lmax = (double)l[ids[t * k]];
+        double sum = 0.0;
+        for (int j = 0; j < k; ++j) {
+            ex[j] = exp((double)l[ids[t * k + j]] - lmax);
+            sum += ex[j];
+        }
+        for (int j = 0; j < k; ++j)
+            weights[t * k + j] = (float)(ex[j] / sum);
+    }
+    free(ex);
+    free(taken);
+}
+
+/* ---- clamped SwiGLU (reading R4; constants from [P3] What it does) ---------- */
+double oracle_swiglu(double gate, double up, double alpha, double limit, int defect)
+{
+    double g = gate, u = up;
+    if (defect != ORACLE_DEFECT_NO_CLAMP) {
+        g = gate < limit ? gate : limit;
+        u = up < -limit ? -limit : (up > limit ? limit : up);
+    }
+    return (u + 1.0) * g / (1.0 + exp(-alpha * g));
+}
+
+/* ---- formulation A: per-token loop, weights decoded on the fly -------------- */
+/* For each listed token t (token_list[r], r < n_list):
+ *   weight on output (flags = 0):
+ *     out[r] = sum_j w[t,j] * ( W_d[e] . act( W_gu[e] . x[t] + b_gu[e] ) + b_d[e] )
+ *   weight on input (flags = ORACLE_FLAG_WEIGHT_ON_INPUT):
+ *     out[r] = sum_j ( W_d[e] . act( W_gu[e] . (w[t,j] x[t]) + b_gu[e] ) + b_d[e] )
+ *   where e = ids[t, j], act splits gate/up (reading R3) and applies the clamped
+ *   SwiGLU.  Biases may be NULL (zero).  [P3] requires both biases absent in the
+ *   weight-on-input mode; the oracle still defines that case the way the review's
+ *   test reference does (biases added unweighted) so that the planted mistake
+ *   ORACLE_DEFECT_WOI_BIAS_WEIGHTED has something to differ from.
+ *   x is bf16 bits [T, H]; W_gu [E, 2I, H] packed; W_d [E, H, I] packed;
+ *   out is double [n_list, H]. */
+void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                           int64_t E, int k, const int32_t *ids, const float *w,
+                           const uint8_t *gu_blocks, const uint8_t *gu_scales,
+                           const float *gu_bias, const uint8_t *d_blocks,
+                           const uint8_t *d_scales, const float *d_bias,
+                           double alpha, double limit, int flags,
+                           const int64_t *token_list, int64_t n_list, double *out,
+                           int defect)
+{
+    (void)T;
+    (void)E;
+    int64_t N_gu = 2 * I;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_list; ++r) {
+        int64_t t = token_list[r];
+        double *xin = (double *)malloc(sizeof(double) * (size_t)H);
+        double *h = (double *)malloc(sizeof(double) * (size_t)N_gu);
+        double *a = (double *)malloc(sizeof(double) * (size_t)I);
+        double *o = out + r * H;
+        for (int64_t c = 0; c < H; ++c)
+            o[c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int64_t e = ids[t * k + j];
+            double wj = (double)w[t * k + j];
+            int woi = (flags & ORACLE_FLAG_WEIGHT_ON_INPUT) != 0;
+            for (int64_t c = 0; c < H; ++c)
+                xin[c] = oracle_bf16_to_double(x[t * H + c]) * (woi ? wj : 1.0);
+            /* gate_up projection with bias before the activation [P3] */
+            for (int64_t n = 0; n < N_gu; ++n) {
+                double acc = 0.0;
+                int zero_row = 0;
+                if (defect == ORACLE_DEFECT_GATE_ZERO)
+                    zero_row = (n % 2) == 0; /* interleaved: even rows are gate */
+                if (!zero_row)
+                    for (int64_t c = 0; c < H; ++c)
+                        acc += xin[c] * weight_elem(gu_blocks, gu_scales, N_gu, H, e, n, c, defect);
+                h[n] = acc + (gu_bias ? (double)gu_bias[e * N_gu + n] : 0.0);
+            }
+            for (int64_t i = 0; i < I; ++i) {
+                double gate, up;
+                if (defect == ORACLE_DEFECT_UNINTERLEAVED) {
+                    gate = h[i];
+                    up = h[I + i];
+                } else {
+                    gate = h[2 * i];
+                    up = h[2 * i + 1];
+                }
+                a[i] = oracle_swiglu(gate, up, alpha, limit, defect);
+            }
+            /* down projection; bias added before the routing weight [P3] */
+            for (int64_t c = 0; c < H; ++c) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < I; ++i)
+                    acc += a[i] * weight_elem(d_blocks, d_scales, H, I, e, c, i, defect);
+                double b = d_bias ? (double)d_bias[e * H + c] : 0.0;
+                if (defect == ORACLE_DEFECT_DOWN_BIAS_IN_SCALE)
+                    b *= oracle_e8m0_value(d_scales[(e * H + c) * (I / 32)], 0);
+                if (woi) {
+                    if (defect == ORACLE_DEFECT_WOI_BIAS_WEIGHTED)
+                        o[c] += acc + wj * b;
+                    else
+                        o[c] += acc + b;
+                } else if (defect == ORACLE_DEFECT_DOWN_BIAS_UNWEIGHTED) {
+                    o[c] += wj * acc + b;
+                } else {
+                    o[c] += wj * (acc + b); /* sum w * (s*y + b), s = 1 for MXFP4 [P3] */
+                }
+            }
+        }
+        free(a);
+        free(h);
+        free(xin);
+    }
+}
+
+/* ---- formulation B: group pairs by expert over a pre-decoded bank ----------- */
+/* Same result as formulation A (up to summation order), computed the way a
+ * grouped kernel organises it: every (token, slot) pair is assigned to its
+ * expert, each expert's pairs go through the expert's two projections as a
+ * small dense matrix product over the fully decoded double-precision bank, and
+ * the rows are scattered back and summed per token in slot order.  Only meant
+ * for small shapes (the decoded bank is E*3*H*I doubles).  No planted mistakes. */
+int oracle_forward_grouped(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                           int64_t E, int k, const int32_t *ids, const float *w,
+                           const uint8_t *gu_blocks, const uint8_t *gu_scales,
+                           const float *gu_bias, const uint8_t *d_blocks,
+                           const uint8_t *d_scales, const float *d_bias,
+                           double alpha, double limit, int flags, double *out)
+{
+    int64_t N_gu = 2 * I;
+    int64_t P = T * k;
+    double *Wgu = (double *)malloc(sizeof(double) * (size_t)(E * N_gu * H));
+    double *Wd = (double *)malloc(sizeof(double) * (size_t)(E * H * I));
+    double *ybuf = (double *)malloc(sizeof(double) * (size_t)(P * H));
+    double *h = (double *)malloc(sizeof(double) * (size_t)N_gu);
+    double *a = (double *)malloc(sizeof(double) * (size_t)I);
+    double *xin = (double *)malloc(sizeof(double) * (size_t)H);
+    if (!Wgu || !Wd || !ybuf || !h || !a || !xin) {
+        free(Wgu); free(Wd); free(ybuf); free(h); free(a); free(xin);
+        return -1;
+    }
+    for (int64_t e = 0; e < E; ++e) {
+        for (int64_t n = 0; n < N_gu; ++n)
+            for (int64_t c = 0; c < H; ++c)
+                Wgu[(e * N_gu + n) * H + c] = weight_elem(gu_blocks, gu_scales, N_gu, H, e, n, c, 0);
+        for (int64_t c = 0; c < H; ++c)
+            for (int64_t i = 0; i < I; ++i)
+                Wd[(e * H + c) * I + i] = weight_elem(d_blocks, d_scales, H, I, e, c, i, 0);
+    }
+    int woi = (flags & ORACLE_FLAG_WEIGHT_ON_INPUT) != 0;
+    for (int64_t e = 0; e < E; ++e) {
+        for (int64_t p = 0; p < P; ++p) { /* pairs p = t*k + j in ascending order */
+            if (ids[p] != e)
+                continue;
+            int64_t t = p / k;
+            double wj = (double)w[p];
+            for (int64_t c = 0; c < H; ++c)
+                xin[c] = oracle_bf16_to_double(x[t * H + c]) * (woi ? wj : 1.0);
+            for (int64_t n = 0; n < N_gu; ++n) {
+                double acc = 0.0;
+                const double *wr = Wgu + (e * N_gu + n) * H;
+                for (int64_t c = 0; c < H; ++c)
+                    acc += wr[c] * xin[c];
+                h[n] = acc + (gu_bias ? (double)gu_bias[e * N_gu + n] : 0.0);
+            }
+            for (int64_t i = 0; i < I; ++i)
+                a[i] = oracle_swiglu(h[2 * i], h[2 * i + 1], alpha, limit, 0);
+            for (int64_t c = 0; c < H; ++c) {
+                double acc = 0.0;
+                const double *wr = Wd + (e * H + c) * I;
+                for (int64_t i = 0; i < I; ++i)
+                    acc += wr[i] * a[i];
+                double y = acc + (d_bias ? (double)d_bias[e * H + c] : 0.0);
+                ybuf[p * H + c] = woi ? y : wj * y;
+            }
+        }
+    }
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < H; ++c) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j)
+                s += ybuf[(t * k + j) * H + c];
+            out[t * H + c] = s;
+        }
+    free(Wgu); free(Wd); free(ybuf); free(h); free(a); free(xin);
+    return 0;
+}
+
+/* Number of OpenMP threads the forward loop may use (1 without OpenMP). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
