@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the MXFP4 expert-FFN MoE layer on B200.
+
+A step is one pass of the layer's hot path over one batch: top-k routing of the
+router logits, then the expert layer (permute, gather, gate_up grouped GEMM with
+clamped SwiGLU, down grouped GEMM with bias and routing weight, combine), all
+through the library's C ABI.  The default workload is the gpt-oss-20b-shaped
+prefill layer (T=4096 tokens, hidden 2880, intermediate 2880, 32 experts, top-4,
+MXFP4 weights) with seeded synthetic inputs.  Secondary measurements (standalone
+dequant, decode, gpt-oss-120b-shaped skewed layers) ride in the same JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank runs an independent replica of the layer
+(the path has no cross-GPU exchange); value = all tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+DEFAULT_WORKLOAD = "20b_prefill_T4096"
+METRIC = "MoE layer tokens/s (prefill)"
+# algorithmic weight bytes of one gpt-oss-20b/120b expert (gate_up + down: packed
+# codes, E8M0 scales, fp32 biases)
+EXPERT_BYTES_2880 = (5760 * 1440 + 5760 * 90 + 5760 * 4) + (2880 * 1440 + 2880 * 90 + 2880 * 4)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-extra", action="store_true", help="skip the secondary measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.device_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
+                "power_w_max": float(max(power)), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- device layer
+
+class DeviceLayer:
+    def __init__(self, layer, device):
+        import torch
+        self.layer = layer
+        self.device = device
+
+        def d(a, dtype=None):
+            if a is None:
+                return None
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            return (t.view(dtype) if dtype is not None else t).to(device)
+
+        self.x = d(layer.x_bits, torch.bfloat16)
+        self.logits = d(layer.logits)
+        self.gu_blocks, self.gu_scales = d(layer.gate_up.blocks), d(layer.gate_up.scales)
+        self.gu_bias = d(layer.gate_up_bias)
+        self.d_blocks, self.d_scales = d(layer.down.blocks), d(layer.down.scales)
+        self.d_bias = d(layer.down_bias)
+        L = layer
+        import mxfp4_expert_ffn_moe_b200 as moe
+        self.moe = moe
+        self.ws = torch.empty(moe.moe_mxfp4_workspace_size(L.T, L.H, L.I, L.E, L.k),
+                              dtype=torch.uint8, device=device)
+        self.ids = torch.empty((L.T, L.k), dtype=torch.int32, device=device)
+        self.w = torch.empty((L.T, L.k), dtype=torch.float32, device=device)
+        self.out = torch.empty((L.T, L.H), dtype=torch.bfloat16, device=device)
+        self.flags = moe.MOE_FLAG_WEIGHT_ON_INPUT if L.weight_on_input else 0
+
+    def step(self, x=None, logits=None):
+        L, moe = self.layer, self.moe
+        moe.moe_route(self.logits if logits is None else logits, L.k, ids=self.ids, weights=self.w)
+        moe.moe_mxfp4_forward_ex(self.x if x is None else x, self.ids, self.w, self.gu_blocks,
+                                 self.gu_scales, self.gu_bias, self.d_blocks, self.d_scales,
+                                 self.d_bias, alpha=L.alpha, limit=L.limit, out=self.out,
+                                 flags=self.flags, workspace=self.ws)
+        return self.out
+
+
+def distinct_experts(logits, k):
+    # count of distinct experts among the top-k of each row (workload statistic)
+    top = np.argsort(-logits, axis=1, kind="stable")[:, :k]
+    return int(np.unique(top).size)
+
+
+def time_steps(fn, steps, stream, flush=None):
+    """Device time (ms) of `steps` calls of fn, with optional L2 flush outside the events."""
+    import torch
+    if flush is None:
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+    total = 0.0
+    evs = []
+    for _ in range(steps):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    for a, b in evs:
+        total += a.elapsed_time(b)
+    return total
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle, timed on this host's cores, on bounded samples of the workload."""
+    import oracle
+    from mxfp4_expert_ffn_moe_b200.workloads import workload
+    oracle.build()
+    layer = workload(args.workload)
+    threads = oracle.num_threads()
+
+    def one_step(n_tok, offset):
+        tokens = (np.arange(n_tok, dtype=np.int64) + offset) % layer.T
+        ids, w = oracle.route(layer.logits[tokens], layer.k)
+        sub_x = layer.x_bits[tokens]
+        oracle.forward_tokens(sub_x, ids, w, layer.gate_up.blocks, layer.gate_up.scales,
+                              layer.gate_up_bias, layer.down.blocks, layer.down.scales,
+                              layer.down_bias, alpha=layer.alpha, limit=layer.limit)
+
+    t0 = time.perf_counter()
+    one_step(threads, 0)
+    t_threads = time.perf_counter() - t0                   # wall time of `threads` tokens
+    budget = 150.0 / max(1, args.steps + args.warmup)      # seconds per step
+    n_tok = max(1, min(threads * 4, int(threads * budget / max(t_threads, 1e-6))))
+    for i in range(args.warmup):
+        one_step(n_tok, 7 * i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one_step(n_tok, 131 * i + 1)
+    dt = time.perf_counter() - t0
+    value = n_tok * args.steps / dt
+    cores = min(threads, n_tok)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "T": layer.T, "H": layer.H, "I": layer.I,
+                   "E": layer.E, "k": layer.k},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} tokens of the {args.workload} layer per step "
+                                   f"(route + forward, decode-on-the-fly double precision)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def cpu_baseline_leg(layer, name):
+    import oracle
+    oracle.build()
+    threads = oracle.num_threads()
+    n_tok = 3 * threads
+    tokens = np.linspace(0, layer.T - 1, n_tok).astype(np.int64)
+    t0 = time.perf_counter()
+    ids, w = oracle.route(layer.logits[tokens], layer.k)
+    oracle.forward_tokens(layer.x_bits[tokens], ids, w, layer.gate_up.blocks, layer.gate_up.scales,
+                          layer.gate_up_bias, layer.down.blocks, layer.down.scales, layer.down_bias,
+                          alpha=layer.alpha, limit=layer.limit)
+    dt = time.perf_counter() - t0
+    return {"value": n_tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_tok} of the {layer.T} tokens of {name} (route + forward), {dt:.1f} s"}
+
+
+def extra_measurements(device, stream, peaks):
+    """Standalone dequant, decode and the gpt-oss-120b-shaped layers (secondary)."""
+    import torch
+    import mxfp4_expert_ffn_moe_b200 as moe
+    from mxfp4_expert_ffn_moe_b200.workloads import make_dequant_bank, workload
+    res = {}
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    # standalone dequant of the gpt-oss-20b expert bank (both projections)
+    gu, dn = make_dequant_bank(seed=0)
+    banks = []
+    nbytes = 0
+    for bank in (gu, dn):
+        E, N, K = bank.shape
+        b = torch.from_numpy(bank.blocks).to(device)
+        s = torch.from_numpy(bank.scales).to(device)
+        o = torch.empty((E, N, K), dtype=torch.bfloat16, device=device)
+        banks.append((b, s, o))
+        nbytes += bank.blocks.nbytes + bank.scales.nbytes + E * N * K * 2
+
+    def deq():
+        for b, s, o in banks:
+            moe.mxfp4_dequantize(b, s, out=o)
+
+    for _ in range(3):
+        deq()
+    moe.moe_profile_read()
+    moe.moe_profile_enable(True)
+    ms = time_steps(deq, 10, stream, flush) / 10
+    prof = moe.moe_profile_read()
+    moe.moe_profile_enable(False)
+    kms = prof["dequant"][0] / max(1, prof["dequant"][1]) * 2
+    res["dequant_20b_bank"] = {
+        "GB/s": nbytes / (ms * 1e-3) / 1e9, "ms": ms, "bytes": nbytes,
+        "kernel_GB/s": nbytes / (kms * 1e-3) / 1e9,
+        "hbm_frac_of_measured": nbytes / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "hbm_frac_of_8TBps": nbytes / (kms * 1e-3) / 1e9 / 8000.0}
+    del banks
+    torch.cuda.empty_cache()
+
+    for name, steps, do_flush in [("20b_decode_T1", 50, True), ("20b_decode_T8", 50, True),
+                                  ("20b_decode_T64", 30, True), ("120b_zipf_T256", 20, True),
+                                  ("120b_zipf_T8192", 5, False)]:
+        layer = workload(name)
+        dl = DeviceLayer(layer, device)
+        for _ in range(3):
+            dl.step()
+        moe.moe_profile_read()
+        moe.moe_profile_enable(True)
+        ms = time_steps(dl.step, steps, stream, flush if do_flush else None) / steps
+        prof = moe.moe_profile_read()
+        moe.moe_profile_enable(False)
+        touched = distinct_experts(layer.logits, layer.k)
+        wbytes = touched * EXPERT_BYTES_2880
+        entry = {"tokens/s": layer.T / (ms * 1e-3), "ms": ms, "touched_experts": touched,
+                 "weight_GB/s": wbytes / (ms * 1e-3) / 1e9,
+                 "hbm_frac_of_measured": wbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                 "stage_ms": {k: v[0] / steps for k, v in prof.items() if v[1]}}
+        flops = 2.0 * layer.T * layer.k * layer.H * 3 * layer.I
+        entry["tflops"] = flops / (ms * 1e-3) / 1e12
+        res[name] = entry
+        del dl
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    from mxfp4_expert_ffn_moe_b200 import build as moe_build
+    if rank == 0:
+        moe_build.build()
+    if world > 1:
+        dist.barrier()
+    import mxfp4_expert_ffn_moe_b200 as moe
+    from mxfp4_expert_ffn_moe_b200.workloads import workload
+    moe.load_library()
+
+    peaks = measured_peaks()
+    layer = workload(args.workload)
+    L = layer
+    dl = DeviceLayer(layer, device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        dl.step()
+    torch.cuda.synchronize()
+    moe.moe_profile_read()
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(uuid) as clocks:
+        moe.moe_profile_enable(True)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            dl.step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        moe.moe_profile_enable(False)
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    prof = moe.moe_profile_read()
+    if world > 1:
+        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    value = world * L.T * args.steps / (ms_total * 1e-3)
+    gpu_launches = sum(v[1] for v in prof.values())
+
+    # end to end through the public API: pinned host inputs -> device -> layer -> host
+    x_host = torch.from_numpy(L.x_bits).view(torch.bfloat16).pin_memory()
+    lg_host = torch.from_numpy(L.logits).pin_memory()
+    out_host = torch.empty((L.T, L.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(dl.x)
+    lg_dev = torch.empty_like(dl.logits)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        lg_dev.copy_(lg_host, non_blocking=True)
+        out = dl.step(x=x_dev, logits=lg_dev)
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = time_steps(e2e_step, e2e_steps, stream)
+    moe.moe_profile_read()
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * L.T * e2e_steps / (e2e_ms * 1e-3)
+
+    # roofline of the dominant kernel (gate_up grouped GEMM), from the live events
+    gu_ms, gu_n = prof["gate_up"]
+    gu_avg = gu_ms / max(1, gu_n)
+    gu_flops = 2.0 * L.T * L.k * L.H * (2 * L.I)
+    achieved = gu_flops / (gu_avg * 1e-3) / 1e12
+    long_region = ms_total > 1000.0
+    peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": "gate_up grouped GEMM",
+                "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_region else 'burst'}",
+                "frac_of_2250_spec": achieved / 2250.0,
+                "flops_per_launch": gu_flops, "avg_launch_ms": gu_avg}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; MXFP4 codes uniform, E8M0 118..126, N(0,1) activations)",
+        "config": {"workload": args.workload, "T": L.T, "H": L.H, "I": L.I, "E": L.E, "k": L.k,
+                   "global_batch": world * L.T, "parallelism": f"replicas x{world}",
+                   "l2": "inputs exceed L2 (424 MB of resident expert weights per step)"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(L.x_bits.nbytes + L.logits.nbytes),
+                "d2h_bytes_per_step": int(L.T * L.H * 2)},
+        "gpu_launches": int(gpu_launches),
+        "stage_ms_per_step": {k: v[0] / args.steps for k, v in prof.items() if v[1]},
+        "roofline": roofline,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_extra:
+        line["extra"] = extra_measurements(device, stream, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(layer, args.workload)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args)
+        return
+    run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

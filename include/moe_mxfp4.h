@@ -1,0 +1,188 @@
+/*
+ * moe_mxfp4.h -- C ABI of the B200 (sm_100a) MXFP4 expert-FFN MoE layer library.
+ *
+ * The layer is the gpt-oss-style mixture-of-experts expert block:
+ *   route:   top-k of the router logits, then a softmax over those k values;
+ *   permute: (token, slot) pairs grouped by expert;
+ *   expert:  h = x . W_gu[e]^T + b_gu[e]  (fp32 accumulate), gate = h[2i],
+ *            up = h[2i+1], a = (clamp(up, -limit, limit) + 1) * g * sigmoid(alpha g)
+ *            with g = min(gate, limit);  y = a . W_d[e]^T + b_d[e];
+ *   combine: out[t] = sum_j w[t,j] * y_j   (the bias sits inside the weight).
+ * Expert weights are MXFP4: E2M1 codes packed two per byte (even element in the
+ * low nibble) with one E8M0 scale byte per 32 consecutive elements of a row.
+ *
+ * Sources, cited by page title and section:
+ *   MoE-Infinity PR #152 "expert offloading Phase 2 -- MXFP4 dequant-on-copy
+ *     execution", Changes: the mxfp4_dequantize op (golden rel-err 0.0) and a
+ *     forward that keeps scales, bias, the [N, K//2] packed layout, the gate/up
+ *     split, clamped SwiGLU and fp32 accumulation.
+ *   FreeToken PR #838 "feat(gguf): serve gpt-oss gguf checkpoints on gpt_oss":
+ *     review "NVFP4 down scale vs. down bias" (sum w*(s*y + b)); review
+ *     "w2_bias with apply_router_weight_on_input" (biases must be absent when the
+ *     router weight scales the input); "What it does" (alpha 1.702, limit 7,
+ *     gate_up_bias [E, 2I], down_bias [E, H], bias before activation / before the
+ *     routing weight).
+ *   onnxruntime/mobius PR #719 "Add native GPT-OSS MXFP4 QMoE export", Summary and
+ *     Validation: blocks [E, N, K/32, 16] (= [E, N, K/2]); E8M0 0x00..0xfe valid,
+ *     0xff rejected.
+ *   transformers PR #49431 "Restore GPT-OSS's router-masked expert-parallel plan":
+ *     MXFP4 experts take routing data (ids + weights) rather than dispatched ids.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are caller-owned DEVICE memory on the current CUDA
+ *     device, contiguous row-major, never freed or retained by the library.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued on it; no call synchronises the host (except
+ *     moe_get_device_error, documented below).
+ *   - Return value: MOE_OK or a negative moe_status.  Argument checks happen on
+ *     the host before anything is enqueued; on an argument error nothing runs and
+ *     no output is touched.  No C++ exception crosses this boundary.
+ *   - Problems only the device can see (an expert id outside [0, E), a 0xff
+ *     scale byte) set a sticky per-device error word read by
+ *     moe_get_device_error; the affected outputs are then unspecified (a 0xff
+ *     scale yields NaN in dequantised values).
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1, /* null pointer, bad size, misalignment, bad flag mix */
+    MOE_ERR_UNSUPPORTED = -2, /* valid but outside what this build implements      */
+    MOE_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed               */
+    MOE_ERR_NO_MEMORY = -4,   /* workspace allocation failed or workspace too small */
+    MOE_ERR_DEVICE = -5       /* the sticky device error word is set                */
+} moe_status;
+
+/* Device error bits reported by moe_get_device_error (ORed). */
+#define MOE_DEVERR_BAD_EXPERT_ID 0x1 /* an id outside [0, E) reached the layer      */
+#define MOE_DEVERR_BAD_SCALE 0x2     /* an E8M0 byte 0xff was decoded                */
+#define MOE_DEVERR_TIMEOUT 0x4       /* a bounded pipeline wait gave up              */
+
+/* moe_mxfp4_forward_ex flags */
+#define MOE_FLAG_WEIGHT_ON_INPUT 0x1u /* router weight scales each expert's input  */
+
+/*
+ * mxfp4_dequantize -- standalone dequant-on-copy of a packed MXFP4 bank to bf16
+ * (MoE-Infinity PR #152, Changes: mxfp4_dequantize; golden rel-err 0.0).
+ *   blocks  uint8  [E, N, K/2]  two E2M1 codes per byte, element 2m in the low
+ *                                nibble of byte m, element 2m+1 in the high nibble
+ *   scales  uint8  [E, N, K/32] E8M0 byte per 32 consecutive elements of a row
+ *   out     bf16   [E, N, K]    out = E2M1(code) * 2^(scale - 127), exact (round
+ *                                to nearest even only where the value is a bf16
+ *                                subnormal or overflows: neither rounds in range);
+ *                                scale 0xff gives NaN and sets MOE_DEVERR_BAD_SCALE
+ * Sizes: E, N >= 1; K >= 32 and K % 32 == 0.  blocks and out must be 16-byte
+ * aligned.  Errors: MOE_ERR_INVALID_ARG for null pointers, sizes or alignment.
+ */
+int mxfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out,
+                     int64_t E, int64_t N, int64_t K, void *stream);
+
+/*
+ * moe_route -- top-k routing (transformers PR #49431: the MXFP4 experts consume
+ * routing ids and weights).  For each token t:
+ *   ids[t, 0..k)     the k largest logits in decreasing order, ties to the lower
+ *                    expert index;
+ *   weights[t, j]    exp(l_j - l_max) / sum over the k chosen of exp(l_i - l_max).
+ *   router_logits fp32 [T, E]; ids int32 [T, k]; weights fp32 [T, k].
+ * Sizes: T >= 1, 1 <= E <= 256, 1 <= k <= min(E, 8).  NaN logits are unsupported.
+ */
+int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *ids,
+              float *weights, void *stream);
+
+/*
+ * moe_mxfp4_forward -- the expert layer, weights on the output
+ * (FreeToken PR #838: sum w*(y + b); bias before the routing weight):
+ *   x               bf16  [T, H]
+ *   ids, weights    int32 / fp32 [T, k]  (e.g. from moe_route)
+ *   gate_up_blocks  uint8 [E, 2I, H/2], gate_up_scales uint8 [E, 2I, H/32]
+ *   gate_up_bias    fp32  [E, 2I] or NULL (= zero)
+ *   down_blocks     uint8 [E, H, I/2],  down_scales uint8 [E, H, I/32]
+ *   down_bias       fp32  [E, H]  or NULL (= zero)
+ *   alpha, limit    clamped SwiGLU constants (gpt-oss: 1.702, 7.0)
+ *   out             bf16  [T, H], must not alias any input
+ * Gate/up rows are interleaved: row 2i of the gate_up bank is gate i, row 2i+1 is
+ * up i.  Sizes: T, E >= 1; 1 <= k <= min(E, 8); H % 64 == 0; I % 64 == 0.
+ * The workspace (moe_mxfp4_workspace_size bytes) is allocated and freed
+ * stream-ordered from the device's default memory pool.
+ */
+int moe_mxfp4_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
+                      const int32_t *ids, const float *weights,
+                      const uint8_t *gate_up_blocks, const uint8_t *gate_up_scales,
+                      const float *gate_up_bias, const uint8_t *down_blocks,
+                      const uint8_t *down_scales, const float *down_bias, float alpha,
+                      float limit, uint16_t *out, void *stream);
+
+/*
+ * moe_mxfp4_forward_ex -- as moe_mxfp4_forward, with flags and a caller workspace.
+ *   flags            0 or MOE_FLAG_WEIGHT_ON_INPUT.  With the router weight on the
+ *                    input each expert sees bf16(w[t,j] * x[t]) and the outputs
+ *                    are summed unweighted; both biases must then be NULL
+ *                    (FreeToken PR #838 review: per-expert biases need the router
+ *                    weight on the output) or MOE_ERR_INVALID_ARG is returned.
+ *   workspace        device memory of at least workspace_bytes, 256-byte aligned,
+ *                    or NULL to let the call allocate it stream-ordered.
+ *   workspace_bytes  >= moe_mxfp4_workspace_size(T, H, I, E, k) when workspace is
+ *                    given, else MOE_ERR_NO_MEMORY.
+ * The workspace must not be used by other work on the GPU while the call runs.
+ */
+int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
+                         const int32_t *ids, const float *weights,
+                         const uint8_t *gate_up_blocks, const uint8_t *gate_up_scales,
+                         const float *gate_up_bias, const uint8_t *down_blocks,
+                         const uint8_t *down_scales, const float *down_bias, float alpha,
+                         float limit, uint16_t *out, uint32_t flags, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace moe_mxfp4_forward_ex needs for these sizes (0 on bad sizes). */
+size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int k);
+
+/* Static English text for a moe_status value. */
+const char *moe_status_string(int status);
+
+/*
+ * moe_get_device_error -- synchronise `stream`, then return the sticky device
+ * error bits (MOE_DEVERR_*) of the current device, clearing them.  Returns a
+ * negative moe_status if the synchronisation itself fails.  Meant for tests and
+ * diagnostics, not for the hot path.
+ */
+int moe_get_device_error(void *stream);
+
+/*
+ * Instrumentation (not part of the layer's math).  Kernel launches made by the
+ * calls above are counted per stage; while timing is enabled each launch is also
+ * bracketed by a pair of CUDA events recorded on the call's stream.
+ *   moe_profile_enable(on)        on != 0 starts event timing, 0 stops it.
+ *   moe_profile_read(ms, launches) waits for every recorded event, writes the
+ *                                 summed kernel milliseconds and the launch counts
+ *                                 per stage (arrays of MOE_PROFILE_STAGES entries,
+ *                                 either may be NULL) since the previous read, and
+ *                                 resets both.  Host-side state, one per process;
+ *                                 not thread-safe.
+ */
+#define MOE_PROFILE_STAGES 7
+enum {
+    MOE_STAGE_ROUTE = 0,   /* moe_route                                   */
+    MOE_STAGE_PERMUTE = 1, /* pair histogram / scan / stable scatter      */
+    MOE_STAGE_GATHER = 2,  /* expert-ordered copy of the inputs           */
+    MOE_STAGE_GATE_UP = 3, /* gate_up grouped GEMM + bias + clamped SwiGLU */
+    MOE_STAGE_DOWN = 4,    /* down grouped GEMM + bias + routing weight   */
+    MOE_STAGE_COMBINE = 5, /* per-token sum of the k expert rows          */
+    MOE_STAGE_DEQUANT = 6  /* mxfp4_dequantize                            */
+};
+int moe_profile_enable(int on);
+int moe_profile_read(double *ms, int64_t *launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,202 @@
+"""B200-native MXFP4 expert-FFN MoE layer: thin Python binding of the C ABI.
+
+The functions below carry the same names as the C entry points declared in
+``include/moe_mxfp4.h`` and only marshal arguments: shapes and raw device pointers
+from torch tensors, the current CUDA stream, and the status code back as an
+exception.  Every step of the layer runs in the CUDA kernels of
+``libmoe_mxfp4.so``; there is no CPU fallback, and calling any function without the
+built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "MoEError", "load_library", "library_path", "mxfp4_dequantize", "moe_route",
+    "moe_mxfp4_forward", "moe_mxfp4_forward_ex", "moe_mxfp4_workspace_size",
+    "moe_status_string", "moe_get_device_error", "MOE_FLAG_WEIGHT_ON_INPUT",
+    "MOE_DEVERR_BAD_EXPERT_ID", "MOE_DEVERR_BAD_SCALE", "MOE_DEVERR_TIMEOUT",
+    "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_read",
+]
+
+MOE_FLAG_WEIGHT_ON_INPUT = 0x1
+MOE_DEVERR_BAD_EXPERT_ID = 0x1
+MOE_DEVERR_BAD_SCALE = 0x2
+MOE_DEVERR_TIMEOUT = 0x4
+
+EXPORTED_SYMBOLS = (
+    "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
+    "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
+    "moe_profile_enable", "moe_profile_read",
+)
+PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {moe_status_string(status)} ({status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libmoe_mxfp4.so")
+
+
+def load_library():
+    """Load the in-tree CUDA library; raise if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    p, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    lib.mxfp4_dequantize.argtypes = [p, p, p, i64, i64, i64, p]
+    lib.mxfp4_dequantize.restype = i32
+    lib.moe_route.argtypes = [p, i64, i64, i32, p, p, p]
+    lib.moe_route.restype = i32
+    fwd = [p, i64, i64, i64, i64, i32, p, p, p, p, p, p, p, p, f32, f32, p]
+    lib.moe_mxfp4_forward.argtypes = fwd + [p]
+    lib.moe_mxfp4_forward.restype = i32
+    lib.moe_mxfp4_forward_ex.argtypes = fwd + [ctypes.c_uint32, p, ctypes.c_size_t, p]
+    lib.moe_mxfp4_forward_ex.restype = i32
+    lib.moe_mxfp4_workspace_size.argtypes = [i64, i64, i64, i64, i32]
+    lib.moe_mxfp4_workspace_size.restype = ctypes.c_size_t
+    lib.moe_status_string.argtypes = [i32]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    lib.moe_get_device_error.argtypes = [p]
+    lib.moe_get_device_error.restype = i32
+    lib.moe_profile_enable.argtypes = [i32]
+    lib.moe_profile_enable.restype = i32
+    lib.moe_profile_read.argtypes = [p, p]
+    lib.moe_profile_read.restype = i32
+    _lib = lib
+    return lib
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    import torch
+    if t is None:
+        return None
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got {t.dtype} "
+                         f"on {t.device} (contiguous={t.is_contiguous()})")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MoEError(fn, rc)
+
+
+def moe_status_string(status: int) -> str:
+    return load_library().moe_status_string(int(status)).decode()
+
+
+def mxfp4_dequantize(blocks, scales, out=None, stream=None):
+    """Packed [E, N, K/2] uint8 + E8M0 [E, N, K/32] uint8 -> bf16 [E, N, K]."""
+    import torch
+    E, N, Kh = blocks.shape
+    K = 2 * Kh
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=blocks.device)
+    rc = load_library().mxfp4_dequantize(_dev(blocks, torch.uint8, "blocks"),
+                                         _dev(scales, torch.uint8, "scales"),
+                                         _dev(out, torch.bfloat16, "out"), E, N, K, _stream(stream))
+    _check("mxfp4_dequantize", rc)
+    return out
+
+
+def moe_route(router_logits, k: int, ids=None, weights=None, stream=None):
+    """fp32 logits [T, E] -> (int32 ids [T, k], fp32 weights [T, k])."""
+    import torch
+    T, E = router_logits.shape
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=router_logits.device)
+    if weights is None:
+        weights = torch.empty((T, k), dtype=torch.float32, device=router_logits.device)
+    rc = load_library().moe_route(_dev(router_logits, torch.float32, "router_logits"), T, E, int(k),
+                                  _dev(ids, torch.int32, "ids"), _dev(weights, torch.float32, "weights"),
+                                  _stream(stream))
+    _check("moe_route", rc)
+    return ids, weights
+
+
+def _fwd_args(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
+              down_scales, down_bias, alpha, limit, out):
+    import torch
+    T, H = x.shape
+    k = ids.shape[1]
+    E, N2, _ = gate_up_blocks.shape
+    I = N2 // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    args = [_dev(x, torch.bfloat16, "x"), T, H, I, E, k, _dev(ids, torch.int32, "ids"),
+            _dev(weights, torch.float32, "weights"), _dev(gate_up_blocks, torch.uint8, "gate_up_blocks"),
+            _dev(gate_up_scales, torch.uint8, "gate_up_scales"),
+            _dev(gate_up_bias, torch.float32, "gate_up_bias"), _dev(down_blocks, torch.uint8, "down_blocks"),
+            _dev(down_scales, torch.uint8, "down_scales"), _dev(down_bias, torch.float32, "down_bias"),
+            float(alpha), float(limit), _dev(out, torch.bfloat16, "out")]
+    return args, out
+
+
+def moe_mxfp4_forward(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
+                      down_scales, down_bias, alpha: float = 1.702, limit: float = 7.0, out=None,
+                      stream=None):
+    args, out = _fwd_args(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias,
+                          down_blocks, down_scales, down_bias, alpha, limit, out)
+    _check("moe_mxfp4_forward", load_library().moe_mxfp4_forward(*args, _stream(stream)))
+    return out
+
+
+def moe_mxfp4_forward_ex(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias,
+                         down_blocks, down_scales, down_bias, alpha: float = 1.702,
+                         limit: float = 7.0, out=None, flags: int = 0, workspace=None,
+                         stream=None):
+    import torch
+    args, out = _fwd_args(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias,
+                          down_blocks, down_scales, down_bias, alpha, limit, out)
+    ws = _dev(workspace, torch.uint8, "workspace")
+    nbytes = 0 if workspace is None else workspace.numel()
+    rc = load_library().moe_mxfp4_forward_ex(*args, ctypes.c_uint32(flags), ws, nbytes, _stream(stream))
+    _check("moe_mxfp4_forward_ex", rc)
+    return out
+
+
+def moe_mxfp4_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(load_library().moe_mxfp4_workspace_size(T, H, I, E, k))
+
+
+def moe_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the sticky device error bits."""
+    rc = load_library().moe_get_device_error(_stream(stream))
+    if rc < 0:
+        raise MoEError("moe_get_device_error", rc)
+    return rc
+
+
+def moe_profile_enable(on: bool = True) -> None:
+    """Start (or stop) CUDA-event timing of every kernel the library launches."""
+    _check("moe_profile_enable", load_library().moe_profile_enable(1 if on else 0))
+
+
+def moe_profile_read():
+    """Per-stage (kernel ms, launch count) since the previous read, as a dict."""
+    n = len(PROFILE_STAGES)
+    ms = (ctypes.c_double * n)()
+    launches = (ctypes.c_int64 * n)()
+    _check("moe_profile_read", load_library().moe_profile_read(ms, launches))
+    return {name: (float(ms[i]), int(launches[i])) for i, name in enumerate(PROFILE_STAGES)}

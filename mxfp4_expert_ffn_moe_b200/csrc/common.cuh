@@ -1,0 +1,48 @@
+// common.cuh -- small device helpers shared by the layer's kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MOE_DEVERR_BAD_EXPERT_ID 0x1
+#define MOE_DEVERR_BAD_SCALE 0x2
+#define MOE_DEVERR_TIMEOUT 0x4
+
+namespace moe {
+
+// Sticky per-device error word (one per loaded module, i.e. per device).
+__device__ int g_device_error;
+
+__device__ __forceinline__ void raise_device_error(int bits) { atomicOr(&g_device_error, bits); }
+
+// fp32 value of an E8M0 scale byte: 2^(s - 127).  s = 0 is the fp32 subnormal
+// 2^-127; s = 0xff is not a number (invalid per the MXFP4 validation rules).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+    if (s == 0u) return __uint_as_float(0x00400000u);
+    if (s == 255u) return __uint_as_float(0x7FC00000u);
+    return __uint_as_float(s << 23);
+}
+
+// Two fp32 values -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Clamped SwiGLU of the gpt-oss expert MLP:
+//   g = min(gate, limit), u = clamp(up, -limit, limit), a = (u + 1) * g * sigmoid(alpha g).
+__device__ __forceinline__ float clamped_swiglu(float gate, float up, float alpha, float limit) {
+    float g = fminf(gate, limit);
+    float u = fminf(fmaxf(up, -limit), limit);
+    float sig = 1.0f / (1.0f + expf(-alpha * g));
+    return (u + 1.0f) * (g * sig);
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace moe

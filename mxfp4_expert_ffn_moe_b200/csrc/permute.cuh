@@ -1,0 +1,119 @@
+// permute.cuh -- group (token, slot) pairs by expert, then gather the expert inputs.
+//
+// Pair p = t*k + j routed to expert ids[p].  The grouped expert GEMMs want the
+// pairs of each expert contiguous ("expert-ordered prefill views", FreeToken PR
+// #838 "What it does"; the "[T, k, 2I] gathers on prefill" of its review), so:
+//   counts[e]        pairs routed to expert e
+//   offsets[e]       first row of expert e in expert order (exclusive scan), offsets[E] = rows
+//   tile_offsets[e]  first M-tile of expert e for an M-tile of bm rows
+//   sorted_pairs[r]  the pair p placed at row r; within an expert rows follow
+//                    ascending p (a stable, deterministic order)
+// Ids outside [0, E) raise MOE_DEVERR_BAD_EXPERT_ID and their pairs are dropped.
+//
+// One CTA of 32 warps: warp w owns a contiguous chunk of pairs, counts its experts
+// in a private shared-memory row, the chunk bases come from an exclusive scan over
+// warps, and each warp then scatters its chunk in order using __match_any_sync to
+// rank equal experts inside a 32-pair step.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermuteThreads = 1024;
+
+__global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
+    const int32_t *__restrict__ ids, int64_t P, int E, int bm, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
+    int32_t *__restrict__ sorted_pairs) {
+    extern __shared__ int sm_perm[];
+    int *cnt = sm_perm;             // [32][E]: per-warp counts, then per-warp running bases
+    int *off = sm_perm + 32 * E;    // [E + 1]: expert start rows
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+
+    const int64_t chunk = (P + 31) / 32;
+    const int64_t beg = (int64_t)warp * chunk;
+    const int64_t end = (beg + chunk < P) ? beg + chunk : P;
+    for (int64_t p = beg + lane; p < end; p += 32) {
+        const int e = ids[p];
+        if ((unsigned)e < (unsigned)E)
+            atomicAdd(&cnt[warp * E + e], 1);
+        else
+            raise_device_error(MOE_DEVERR_BAD_EXPERT_ID);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < 32; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
+        off[e] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0, trun = 0;
+        for (int e = 0; e < E; ++e) {
+            const int c = off[e];
+            counts[e] = c;
+            offsets[e] = run;
+            tile_offsets[e] = trun;
+            off[e] = run;
+            run += c;
+            trun += (c + bm - 1) / bm;
+        }
+        offsets[E] = run;
+        tile_offsets[E] = trun;
+        off[E] = run;
+    }
+    __syncthreads();
+    for (int64_t base = beg; base < end; base += 32) {
+        const int64_t p = base + lane;
+        const int e = (p < end) ? ids[p] : -1;
+        const bool valid = (p < end) && (unsigned)e < (unsigned)E;
+        const int key = valid ? e : -1 - lane;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int wbase = valid ? cnt[warp * E + e] : 0;
+        __syncwarp();
+        if (valid) {
+            sorted_pairs[off[e] + wbase + rank] = (int32_t)p;
+            if (rank == 0) cnt[warp * E + e] = wbase + __popc(peers);
+        }
+        __syncwarp();
+    }
+}
+
+// x_perm[r] = x[t] (router weight on the output) or bf16(w[p] * x[t]) (router
+// weight on the input), t = sorted_pairs[r] / k.  One warp per row, 16-byte chunks.
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const uint16_t *__restrict__ x, const float *__restrict__ weights,
+    const int32_t *__restrict__ sorted_pairs, const int32_t *__restrict__ offsets, int E, int k,
+    int64_t H, int weight_on_input, uint16_t *__restrict__ x_perm) {
+    const int rows = offsets[E];
+    const int lane = threadIdx.x & 31;
+    const int wpb = blockDim.x >> 5;
+    const int64_t chunks = H / 8;
+    for (int64_t r = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); r < rows;
+         r += (int64_t)gridDim.x * wpb) {
+        const int p = sorted_pairs[r];
+        const int64_t t = p / k;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
+        const float w = weight_on_input ? weights[p] : 1.0f;
+        for (int64_t c = lane; c < chunks; c += 32) {
+            uint4 v = __ldg(src + c);
+            if (weight_on_input) {
+                v.x = pack_bf16x2(bf16lo_to_f32(v.x) * w, bf16hi_to_f32(v.x) * w);
+                v.y = pack_bf16x2(bf16lo_to_f32(v.y) * w, bf16hi_to_f32(v.y) * w);
+                v.z = pack_bf16x2(bf16lo_to_f32(v.z) * w, bf16hi_to_f32(v.z) * w);
+                v.w = pack_bf16x2(bf16lo_to_f32(v.w) * w, bf16hi_to_f32(v.w) * w);
+            }
+            dst[c] = v;
+        }
+    }
+}
+
+}  // namespace moe

@@ -17,3 +17,17 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def moe_gpu():
+    """The CUDA library, built in-tree if needed, on a visible GPU."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    from mxfp4_expert_ffn_moe_b200 import build as moe_build
+    moe_build.build()
+    import mxfp4_expert_ffn_moe_b200 as moe
+    moe.load_library()
+    moe.moe_get_device_error()  # start from a clear error word
+    return moe

@@ -1,0 +1,65 @@
+"""Helpers for the GPU tests: move seeded workload arrays to the device and run
+the layer through the C ABI (via the package binding).  No layer arithmetic."""
+import numpy as np
+
+
+def to_dev(a, dtype=None):
+    import torch
+    if a is None:
+        return None
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+def layer_to_device(layer):
+    import torch
+    return dict(
+        x=to_dev(layer.x_bits, torch.bfloat16),
+        logits=to_dev(layer.logits),
+        gu_blocks=to_dev(layer.gate_up.blocks), gu_scales=to_dev(layer.gate_up.scales),
+        gu_bias=to_dev(layer.gate_up_bias),
+        d_blocks=to_dev(layer.down.blocks), d_scales=to_dev(layer.down.scales),
+        d_bias=to_dev(layer.down_bias),
+    )
+
+
+def bf16_tensor_to_f64(t):
+    import torch
+    bits = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def bits_of(t):
+    import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_forward(moe, dev, ids, w, layer, flags=None, workspace=None):
+    import torch
+    ids_d = ids if isinstance(ids, torch.Tensor) else to_dev(ids.astype(np.int32))
+    w_d = w if isinstance(w, torch.Tensor) else to_dev(w.astype(np.float32))
+    if flags is None:
+        flags = moe.MOE_FLAG_WEIGHT_ON_INPUT if layer.weight_on_input else 0
+    out = moe.moe_mxfp4_forward_ex(dev["x"], ids_d, w_d, dev["gu_blocks"], dev["gu_scales"],
+                                   dev["gu_bias"], dev["d_blocks"], dev["d_scales"], dev["d_bias"],
+                                   alpha=layer.alpha, limit=layer.limit, flags=flags,
+                                   workspace=workspace)
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_forward(oracle, layer, ids, w, tokens=None):
+    return oracle.forward_tokens(layer.x_bits, ids, w, layer.gate_up.blocks, layer.gate_up.scales,
+                                 layer.gate_up_bias, layer.down.blocks, layer.down.scales,
+                                 layer.down_bias, alpha=layer.alpha, limit=layer.limit,
+                                 weight_on_input=layer.weight_on_input, tokens=tokens)
+
+
+def sample_tokens(T, n, seed=0):
+    if T <= n:
+        return np.arange(T, dtype=np.int64)
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
+    return np.sort(np.concatenate([[0, T - 1], mid])).astype(np.int64)

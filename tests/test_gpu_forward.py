@@ -1,0 +1,146 @@
+"""moe_mxfp4_forward on the GPU against the CPU oracle.
+
+Layer output tolerance (bf16 output vs the double-precision oracle): relative L2
+error <= 1e-2 and max |error| <= 2e-2 * RMS(oracle output).  Small cases are
+compared in full; full-size workloads on sampled tokens (every token is computed
+on the GPU, the oracle evaluates the sampled ones one by one).
+"""
+import numpy as np
+import pytest
+
+from mxfp4_expert_ffn_moe_b200.workloads import make_layer, workload
+from tests._metrics import MAX_ABS_OVER_RMS_TOL, REL_L2_TOL, max_abs_over_rms, rel_l2
+from tests.gpu_util import (bf16_tensor_to_f64, layer_to_device, oracle_forward, run_forward,
+                            sample_tokens, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+def _assert_close(got, want, what=""):
+    """The stated layer tolerance, used for every configured workload."""
+    r, m = rel_l2(got, want), max_abs_over_rms(got, want)
+    assert r <= REL_L2_TOL and m <= MAX_ABS_OVER_RMS_TOL, f"{what}: rel_l2={r:.3g} max/rms={m:.3g}"
+
+
+# Rounding a value v to the bf16 output alone moves it by up to half an ulp,
+# 2^-8 |v|.  Once max|out| exceeds about 5x RMS(out) that by itself can pass
+# 2e-2 * RMS, so the extra edge shapes (heavy-tailed outputs: small H or I, unit
+# biases) are held to the stated bound on top of the output format's own rounding:
+#   |got - want| <= 2e-2 * RMS(want) + 2^-8 |want|   elementwise, rel-L2 <= 1e-2.
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
+def _assert_close_bf16_output(got, want, what=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    rms = float(np.sqrt(np.mean(want * want)))
+    excess = np.abs(got - want) - BF16_HALF_ULP_REL * np.abs(want)
+    r = rel_l2(got, want)
+    m = float(np.max(excess)) / rms
+    assert r <= REL_L2_TOL and m <= MAX_ABS_OVER_RMS_TOL, f"{what}: rel_l2={r:.3g} excess/rms={m:.3g}"
+
+
+def _check_layer(moe, oracle, layer, n_sample=None, seed=0, check=_assert_close):
+    dev = layer_to_device(layer)
+    ids, w = oracle.route(layer.logits, layer.k)
+    out = run_forward(moe, dev, ids, w, layer)
+    got = bf16_tensor_to_f64(out)
+    tokens = sample_tokens(layer.T, n_sample or layer.T, seed)
+    want = oracle_forward(oracle, layer, ids, w, tokens)
+    check(got[tokens], want, layer.name)
+    assert moe.moe_get_device_error() == 0
+    return got
+
+
+@pytest.mark.parametrize("name", ["tiny_woo", "tiny_woi", "tiny_bias_heavy"])
+def test_tiny_layers_full_compare(moe_gpu, oracle_mod, name):
+    _check_layer(moe_gpu, oracle_mod, workload(name))
+
+
+@pytest.mark.parametrize("T,H,I,E,k,woi", [
+    (1, 64, 64, 1, 1, False),        # dense MLP, single token
+    (37, 192, 320, 5, 3, False),     # ragged M tiles, several N tiles, empty experts likely
+    (130, 128, 64, 3, 2, True),      # more than two M tiles per expert, weight on input
+    (3, 256, 128, 16, 4, False),     # most experts empty
+    (200, 64, 128, 2, 2, False),     # every pair on the same two experts
+])
+def test_edge_shapes(moe_gpu, oracle_mod, T, H, I, E, k, woi):
+    layer = make_layer(T, H, I, E, k, seed=T + H, biases=not woi, weight_on_input=woi,
+                       bias_std=1.0, name=f"edge_{T}_{H}_{I}_{E}_{k}")
+    _check_layer(moe_gpu, oracle_mod, layer, check=_assert_close_bf16_output)
+
+
+@pytest.mark.parametrize("name,n_sample", [
+    ("20b_decode_T1", 1), ("20b_decode_T8", 8), ("20b_decode_T64", 16),
+    ("20b_prefill_T4096", 24), ("120b_zipf_T256", 16), ("120b_zipf_T8192", 24),
+])
+def test_full_size_workloads_sampled(moe_gpu, oracle_mod, name, n_sample):
+    _check_layer(moe_gpu, oracle_mod, workload(name), n_sample=n_sample)
+
+
+def test_route_then_forward_end_to_end(moe_gpu, oracle_mod):
+    import torch
+    layer = workload("20b_decode_T64")
+    dev = layer_to_device(layer)
+    ids_d, w_d = moe_gpu.moe_route(dev["logits"], layer.k)
+    out = run_forward(moe_gpu, dev, ids_d, w_d, layer)
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    np.testing.assert_array_equal(ids_d.cpu().numpy(), ids)
+    tokens = sample_tokens(layer.T, 8, 3)
+    _assert_close(bf16_tensor_to_f64(out)[tokens], oracle_forward(oracle_mod, layer, ids, w, tokens))
+    torch.cuda.synchronize()
+
+
+def test_deterministic_and_caller_workspace(moe_gpu, oracle_mod):
+    import torch
+    layer = workload("tiny_bias_heavy")
+    dev = layer_to_device(layer)
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    a = run_forward(moe_gpu, dev, ids, w, layer)
+    b = run_forward(moe_gpu, dev, ids, w, layer)
+    nbytes = moe_gpu.moe_mxfp4_workspace_size(layer.T, layer.H, layer.I, layer.E, layer.k)
+    ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")
+    c = run_forward(moe_gpu, dev, ids, w, layer, workspace=ws)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+
+
+def test_weight_on_input_with_bias_is_refused(moe_gpu):
+    layer = workload("tiny_woo")
+    dev = layer_to_device(layer)
+    ids = np.zeros((layer.T, layer.k), np.int32)
+    w = np.ones((layer.T, layer.k), np.float32)
+    with pytest.raises(moe_gpu.MoEError) as ei:
+        run_forward(moe_gpu, dev, ids, w, layer, flags=moe_gpu.MOE_FLAG_WEIGHT_ON_INPUT)
+    assert ei.value.status == -1
+
+
+def test_bad_expert_id_sets_device_error(moe_gpu, oracle_mod):
+    layer = workload("tiny_woo")
+    dev = layer_to_device(layer)
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    bad_ids = ids.copy()
+    bad_ids[3, 1] = layer.E + 5
+    out = run_forward(moe_gpu, dev, bad_ids, w, layer)
+    assert moe_gpu.moe_get_device_error() & moe_gpu.MOE_DEVERR_BAD_EXPERT_ID
+    # the dropped slot contributes nothing; every other slot is intact
+    w_ref = w.copy()
+    w_ref[3, 1] = 0.0
+    ids_ref = ids.copy()
+    ids_ref[3, 1] = 0
+    want = oracle_forward(oracle_mod, layer, ids_ref, w_ref)
+    _assert_close(bf16_tensor_to_f64(out), want)
+
+
+def test_invalid_scale_byte_gives_nan_and_flag(moe_gpu, oracle_mod):
+    import torch
+    layer = workload("tiny_woo")
+    scales = layer.down.scales.copy()
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    e = int(ids[0, 0])
+    scales[e, 0, 0] = 255
+    dev = layer_to_device(layer)
+    dev["d_scales"] = to_dev(scales)
+    out = run_forward(moe_gpu, dev, ids, w, layer)
+    assert moe_gpu.moe_get_device_error() & moe_gpu.MOE_DEVERR_BAD_SCALE
+    assert torch.isnan(out.float()[0, 0]).item()

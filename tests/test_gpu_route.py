@@ -1,0 +1,39 @@
+"""moe_route on the GPU against the CPU oracle: ids bit-exact, weights to fp32 rounding."""
+import numpy as np
+import pytest
+
+from mxfp4_expert_ffn_moe_b200.workloads import workload
+from tests.gpu_util import to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _route(moe, logits, k):
+    import torch
+    ids, w = moe.moe_route(to_dev(logits), k)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 4, 1), (8, 4, 2), (37, 32, 4), (4096, 32, 4),
+                                   (300, 128, 4), (65, 200, 8), (5, 256, 8), (9, 7, 7)])
+def test_route_matches_oracle(moe_gpu, oracle_mod, T, E, k):
+    rng = np.random.default_rng(T * 7 + E)
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    logits[0, :] = 0.25                       # a fully tied row
+    if T > 2:
+        logits[2, ::3] = logits[2, 1]         # partial ties
+    ids, w = _route(moe_gpu, logits, k)
+    ids_o, w_o = oracle_mod.route(logits, k)
+    np.testing.assert_array_equal(ids, ids_o)
+    np.testing.assert_allclose(w, w_o, rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(w.astype(np.float64).sum(axis=1), 1.0, atol=1e-6)
+
+
+@pytest.mark.parametrize("name", ["20b_prefill_T4096", "120b_zipf_T8192"])
+def test_route_full_size_workloads(moe_gpu, oracle_mod, name):
+    layer = workload(name)
+    ids, w = _route(moe_gpu, layer.logits, layer.k)
+    ids_o, w_o = oracle_mod.route(layer.logits, layer.k)
+    np.testing.assert_array_equal(ids, ids_o)
+    np.testing.assert_allclose(w, w_o, rtol=1e-6, atol=1e-7)
