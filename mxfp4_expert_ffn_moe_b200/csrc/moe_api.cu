@@ -9,11 +9,14 @@
 
 #include <vector>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "../../include/moe_mxfp4.h"
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
-#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -99,6 +102,82 @@ int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n > 0 ? n : 148;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// bf16 activations [rows, K], K-major: box of 64 elements (128 B, swizzled) x BM rows.
+bool make_act_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)moe::tc::BK, (cuuint32_t)moe::tc::BM};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// packed MXFP4 codes [E, N, K/2] bytes: box of 32 bytes (64 codes) x BN rows x 1 expert.
+bool make_weight_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
+    cuuint32_t box[3] = {(cuuint32_t)(moe::tc::BK / 2), (cuuint32_t)moe::tc::BN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kGateUp>
+int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, const uint8_t *wblocks,
+                        const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
+                        const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
+                        uint16_t *act, float alpha, float limit, float *yp,
+                        const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
+    CUtensorMap ma, mw;
+    if (!make_act_map(&ma, A, rows, K) || !make_weight_map(&mw, wblocks, E, N, K)) return MOE_ERR_CUDA;
+    if (cudaFuncSetAttribute(moe::tc::grouped_mxfp4_tc_kernel<kGateUp>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)moe::tc::SMEM_BYTES) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    moe::tc::Params p{};
+    p.counts = counts;
+    p.offsets = offsets;
+    p.tile_offsets = tile_offsets;
+    p.wscales = wscales;
+    p.bias = bias;
+    p.E = (int)E;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.act = act;
+    p.alpha = alpha;
+    p.limit = limit;
+    p.yp = yp;
+    p.sorted_pairs = sorted_pairs;
+    p.weights = weights;
+    p.weight_on_input = woi;
+    const int64_t n_tiles = moe::ceil_div(N, moe::tc::BN);
+    const int64_t max_tiles = (moe::ceil_div(rows, moe::tc::BM) + E) * n_tiles;
+    const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
+    StageScope scope(stage, s);
+    moe::tc::grouped_mxfp4_tc_kernel<kGateUp>
+        <<<grid, moe::tc::kThreads, moe::tc::SMEM_BYTES, s>>>(ma, mw, p);
+    return launch_check();
 }
 
 }  // namespace
@@ -214,7 +293,7 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
             const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
             StageScope sp(MOE_STAGE_PERMUTE, s);
             moe::permute_pairs_kernel<<<1, moe::kPermuteThreads, perm_smem, s>>>(
-                ids, P, (int)E, moe::kSimtBM, counts, offsets, tile_offsets, sorted_pairs);
+                ids, P, (int)E, moe::tc::BM, counts, offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
         {
@@ -224,23 +303,16 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                 x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
         }
         if ((rc = launch_check()) != MOE_OK) break;
-        const int64_t mtiles = moe::ceil_div(P, moe::kSimtBM) + E;
-        {
-            dim3 g1((unsigned)mtiles, (unsigned)((2 * I) / moe::kSimtBN));
-            StageScope su(MOE_STAGE_GATE_UP, s);
-            moe::grouped_mxfp4_simt_kernel<true><<<g1, 256, 0, s>>>(
-                x_perm, gate_up_blocks, gate_up_scales, gate_up_bias, counts, offsets, tile_offsets,
-                (int)E, (int)(2 * I), (int)H, act, alpha, limit, nullptr, sorted_pairs, weights, 0);
-        }
-        if ((rc = launch_check()) != MOE_OK) break;
-        {
-            dim3 g2((unsigned)mtiles, (unsigned)(H / moe::kSimtBN));
-            StageScope sd(MOE_STAGE_DOWN, s);
-            moe::grouped_mxfp4_simt_kernel<false><<<g2, 256, 0, s>>>(
-                act, down_blocks, down_scales, down_bias, counts, offsets, tile_offsets, (int)E,
-                (int)H, (int)I, nullptr, alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0);
-        }
-        if ((rc = launch_check()) != MOE_OK) break;
+        if ((rc = launch_grouped_gemm<true>(MOE_STAGE_GATE_UP, x_perm, P, H, gate_up_blocks,
+                                            gate_up_scales, gate_up_bias, E, 2 * I, counts, offsets,
+                                            tile_offsets, act, alpha, limit, nullptr, sorted_pairs,
+                                            weights, 0, s)) != MOE_OK)
+            break;
+        if ((rc = launch_grouped_gemm<false>(MOE_STAGE_DOWN, act, P, I, down_blocks, down_scales,
+                                             down_bias, E, H, counts, offsets, tile_offsets, nullptr,
+                                             alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0,
+                                             s)) != MOE_OK)
+            break;
         {
             const int64_t n4 = T * (H / 4);
             const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;

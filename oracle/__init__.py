@@ -81,7 +81,7 @@ def _load():
         lib.oracle_forward_tokens.restype = None
         lib.oracle_forward_tokens.argtypes = [p, i64, i64, i64, i64, ctypes.c_int, p, p,
                                               p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
-                                              ctypes.c_int, p, i64, p, ctypes.c_int]
+                                              ctypes.c_int, p, i64, p, p, ctypes.c_int]
         lib.oracle_forward_grouped.restype = ctypes.c_int
         lib.oracle_forward_grouped.argtypes = [p, i64, i64, i64, i64, ctypes.c_int, p, p,
                                                p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
@@ -143,8 +143,9 @@ def route(logits, k: int):
 
 def forward_tokens(x_bits, ids, weights, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,
                    d_bias, alpha=1.702, limit=7.0, weight_on_input=False, tokens=None,
-                   defect: int = DEFECT_NONE) -> np.ndarray:
-    """Formulation A.  x_bits: bf16 bits uint16 [T,H].  Returns float64 [len(tokens), H]."""
+                   defect: int = DEFECT_NONE, envelope: bool = False):
+    """Formulation A.  x_bits: bf16 bits uint16 [T,H].  Returns float64 [len(tokens), H],
+    or (out, env) with the down projection's magnitude envelope when envelope=True."""
     x_bits = _c(x_bits, np.uint16)
     T, H = x_bits.shape
     ids = _c(ids, np.int32)
@@ -157,13 +158,14 @@ def forward_tokens(x_bits, ids, weights, gu_blocks, gu_scales, gu_bias, d_blocks
         tokens = np.arange(T, dtype=np.int64)
     tokens = _c(tokens, np.int64)
     out = np.empty((tokens.size, H), dtype=np.float64)
+    env = np.empty((tokens.size, H), dtype=np.float64) if envelope else None
     _load().oracle_forward_tokens(
         _ptr(x_bits), T, H, I, E, k, _ptr(ids), _ptr(weights), _ptr(gu_blocks),
         _ptr(_c(gu_scales, np.uint8)), _ptr(_c(gu_bias, np.float32)), _ptr(_c(d_blocks, np.uint8)),
         _ptr(_c(d_scales, np.uint8)), _ptr(_c(d_bias, np.float32)), float(alpha), float(limit),
         FLAG_WEIGHT_ON_INPUT if weight_on_input else 0, _ptr(tokens), tokens.size, _ptr(out),
-        int(defect))
-    return out
+        _ptr(env), int(defect))
+    return (out, env) if envelope else out
 
 
 def forward_grouped(x_bits, ids, weights, gu_blocks, gu_scales, gu_bias, d_blocks, d_scales,

@@ -218,7 +218,13 @@ double oracle_swiglu(double gate, double up, double alpha, double limit, int def
  *   test reference does (biases added unweighted) so that the planted mistake
  *   ORACLE_DEFECT_WOI_BIAS_WEIGHTED has something to differ from.
  *   x is bf16 bits [T, H]; W_gu [E, 2I, H] packed; W_d [E, H, I] packed;
- *   out is double [n_list, H]. */
+ *   out is double [n_list, H].
+ *   env (optional, may be NULL) receives the magnitude envelope of the down
+ *   projection, the sum over j of |w_eff| * (sum_i |a_i * W_d[e, c, i]| + |b_d[e, c]|)
+ *   with w_eff the routing weight applied to that slot's output (1 with the weight on
+ *   the input).  It bounds |out| by the triangle inequality and scales the error a
+ *   rounded activation operand can cause (MoE-Infinity PR #152, Changes: the parity
+ *   test pairs an fp32 golden with a magnitude envelope). */
 void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
                            int64_t E, int k, const int32_t *ids, const float *w,
                            const uint8_t *gu_blocks, const uint8_t *gu_scales,
@@ -226,7 +232,7 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
                            const uint8_t *d_scales, const float *d_bias,
                            double alpha, double limit, int flags,
                            const int64_t *token_list, int64_t n_list, double *out,
-                           int defect)
+                           double *env, int defect)
 {
     (void)T;
     (void)E;
@@ -238,8 +244,12 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
         double *h = (double *)malloc(sizeof(double) * (size_t)N_gu);
         double *a = (double *)malloc(sizeof(double) * (size_t)I);
         double *o = out + r * H;
-        for (int64_t c = 0; c < H; ++c)
+        double *ev = env ? env + r * H : NULL;
+        for (int64_t c = 0; c < H; ++c) {
             o[c] = 0.0;
+            if (ev)
+                ev[c] = 0.0;
+        }
         for (int j = 0; j < k; ++j) {
             int64_t e = ids[t * k + j];
             double wj = (double)w[t * k + j];
@@ -270,10 +280,15 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
             }
             /* down projection; bias added before the routing weight [P3] */
             for (int64_t c = 0; c < H; ++c) {
-                double acc = 0.0;
-                for (int64_t i = 0; i < I; ++i)
-                    acc += a[i] * weight_elem(d_blocks, d_scales, H, I, e, c, i, defect);
+                double acc = 0.0, mag = 0.0;
+                for (int64_t i = 0; i < I; ++i) {
+                    double term = a[i] * weight_elem(d_blocks, d_scales, H, I, e, c, i, defect);
+                    acc += term;
+                    mag += fabs(term);
+                }
                 double b = d_bias ? (double)d_bias[e * H + c] : 0.0;
+                if (ev)
+                    ev[c] += (woi ? 1.0 : fabs(wj)) * (mag + fabs(b));
                 if (defect == ORACLE_DEFECT_DOWN_BIAS_IN_SCALE)
                     b *= oracle_e8m0_value(d_scales[(e * H + c) * (I / 32)], 0);
                 if (woi) {

@@ -50,11 +50,12 @@ def run_forward(moe, dev, ids, w, layer, flags=None, workspace=None):
     return out
 
 
-def oracle_forward(oracle, layer, ids, w, tokens=None):
+def oracle_forward(oracle, layer, ids, w, tokens=None, envelope=False):
     return oracle.forward_tokens(layer.x_bits, ids, w, layer.gate_up.blocks, layer.gate_up.scales,
                                  layer.gate_up_bias, layer.down.blocks, layer.down.scales,
                                  layer.down_bias, alpha=layer.alpha, limit=layer.limit,
-                                 weight_on_input=layer.weight_on_input, tokens=tokens)
+                                 weight_on_input=layer.weight_on_input, tokens=tokens,
+                                 envelope=envelope)
 
 
 def sample_tokens(T, n, seed=0):

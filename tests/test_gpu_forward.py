@@ -22,32 +22,39 @@ def _assert_close(got, want, what=""):
     assert r <= REL_L2_TOL and m <= MAX_ABS_OVER_RMS_TOL, f"{what}: rel_l2={r:.3g} max/rms={m:.3g}"
 
 
-# Rounding a value v to the bf16 output alone moves it by up to half an ulp,
-# 2^-8 |v|.  Once max|out| exceeds about 5x RMS(out) that by itself can pass
-# 2e-2 * RMS, so the extra edge shapes (heavy-tailed outputs: small H or I, unit
-# biases) are held to the stated bound on top of the output format's own rounding:
-#   |got - want| <= 2e-2 * RMS(want) + 2^-8 |want|   elementwise, rel-L2 <= 1e-2.
-BF16_HALF_ULP_REL = 2.0 ** -8
+# Extra edge shapes (small H or I, unit biases, heavy-tailed outputs) get a bound
+# derived from the arithmetic instead of the configured one.  Rounding the output to
+# bf16 moves a value v by up to half an ulp, 2^-8 |v|; rounding each activation a_i
+# (and, with the weight on the input, each w*x) to the bf16 MMA operand moves the
+# down projection by at most 2^-9 sum_i |a_i W_i| per rounding, i.e. within 2^-8 of
+# the magnitude envelope env the oracle reports (the fp32-golden plus
+# magnitude-envelope parity test of MoE-Infinity PR #152).  So, elementwise,
+#   |got - want| <= 2e-2 * RMS(want) + 2^-8 |want| + 2^-8 env,   rel-L2 <= 1e-2.
+# With max|out| near 10x RMS the first term alone cannot absorb these roundings.
+BF16_U2 = 2.0 ** -8
 
 
-def _assert_close_bf16_output(got, want, what=""):
+def _assert_close_envelope(got, want, env, what=""):
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
     rms = float(np.sqrt(np.mean(want * want)))
-    excess = np.abs(got - want) - BF16_HALF_ULP_REL * np.abs(want)
+    excess = np.abs(got - want) - BF16_U2 * (np.abs(want) + env)
     r = rel_l2(got, want)
     m = float(np.max(excess)) / rms
     assert r <= REL_L2_TOL and m <= MAX_ABS_OVER_RMS_TOL, f"{what}: rel_l2={r:.3g} excess/rms={m:.3g}"
 
 
-def _check_layer(moe, oracle, layer, n_sample=None, seed=0, check=_assert_close):
+def _check_layer(moe, oracle, layer, n_sample=None, seed=0, envelope=False):
     dev = layer_to_device(layer)
     ids, w = oracle.route(layer.logits, layer.k)
     out = run_forward(moe, dev, ids, w, layer)
     got = bf16_tensor_to_f64(out)
     tokens = sample_tokens(layer.T, n_sample or layer.T, seed)
-    want = oracle_forward(oracle, layer, ids, w, tokens)
-    check(got[tokens], want, layer.name)
+    if envelope:
+        want, env = oracle_forward(oracle, layer, ids, w, tokens, envelope=True)
+        _assert_close_envelope(got[tokens], want, env, layer.name)
+    else:
+        _assert_close(got[tokens], oracle_forward(oracle, layer, ids, w, tokens), layer.name)
     assert moe.moe_get_device_error() == 0
     return got
 
@@ -67,7 +74,7 @@ def test_tiny_layers_full_compare(moe_gpu, oracle_mod, name):
 def test_edge_shapes(moe_gpu, oracle_mod, T, H, I, E, k, woi):
     layer = make_layer(T, H, I, E, k, seed=T + H, biases=not woi, weight_on_input=woi,
                        bias_std=1.0, name=f"edge_{T}_{H}_{I}_{E}_{k}")
-    _check_layer(moe_gpu, oracle_mod, layer, check=_assert_close_bf16_output)
+    _check_layer(moe_gpu, oracle_mod, layer, envelope=True)
 
 
 @pytest.mark.parametrize("name,n_sample", [

@@ -397,3 +397,25 @@ def test_planted_woi_bias_mistake_is_caught(oracle_mod):
                                     defect=oracle_mod.DEFECT_WOI_BIAS_WEIGHTED)
     # biases are small (N(0, 0.02)); the mistake must still be visible per element
     assert np.max(np.abs(bad - good)) > 1e-3
+
+
+def test_envelope_bounds_output_and_matches_dense_special_case(oracle_mod, tiny_woo):
+    # Triangle inequality: |out| <= env elementwise.
+    layer = tiny_woo
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    out, env = oracle_mod.forward_tokens(*_args(layer, ids, w), envelope=True)
+    assert np.all(np.abs(out) <= env * (1 + 1e-12))
+    np.testing.assert_array_equal(out, oracle_mod.forward_tokens(*_args(layer, ids, w)))
+    # Dense special case (E = k = 1, w = 1): env = |W_d| @ |a| + |b_d| with numpy.
+    layer = make_layer(T=4, H=64, I=96, E=1, k=1, seed=21)
+    ids1 = np.zeros((4, 1), np.int32)
+    w1 = np.ones((4, 1), np.float32)
+    _, env = oracle_mod.forward_tokens(*_args(layer, ids1, w1), envelope=True)
+    H, I = layer.H, layer.I
+    Wgu = bf16_bits_to_f32(oracle_mod.dequantize(layer.gate_up.blocks, layer.gate_up.scales, 1, 2 * I, H))[0]
+    Wd = bf16_bits_to_f32(oracle_mod.dequantize(layer.down.blocks, layer.down.scales, 1, H, I))[0]
+    x = bf16_bits_to_f32(layer.x_bits).astype(np.float64)
+    h = x @ Wgu.astype(np.float64).T + layer.gate_up_bias[0].astype(np.float64)
+    act = np.vectorize(oracle_mod.swiglu)(h[:, 0::2], h[:, 1::2])
+    want = np.abs(act) @ np.abs(Wd.astype(np.float64)).T + np.abs(layer.down_bias[0].astype(np.float64))
+    assert rel_l2(env, want) < 1e-12
