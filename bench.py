@@ -39,7 +39,7 @@ EXPERT_BYTES_2880 = (5760 * 1440 + 5760 * 90 + 5760 * 4) + (2880 * 1440 + 2880 *
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
@@ -63,7 +63,7 @@ def measured_peaks():
 
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons while it runs."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -71,6 +71,11 @@ class ClockSampler:
         self.device_id = device_id
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.window = None
+
+    def mark(self, t0: float, t1: float):
+        """Wall-clock bounds (time.time()) of the timed region."""
+        self.window = (t0, t1)
 
     def __enter__(self):
         try:
@@ -94,25 +99,33 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
+        import datetime
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         sm, smax, reasons, power = [], [], set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        n_all = 0
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
+            if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-                power.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                vals = float(parts[1]), float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[4:8]):
+            n_all += 1
+            if self.window and not (self.window[0] - 0.05 <= ts <= self.window[1] + 0.05):
+                continue
+            sm.append(vals[0])
+            smax.append(vals[1])
+            power.append(vals[2])
+            for n, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"no samples in the timed "
+                                                                     f"window ({n_all} outside)"]}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)),
                 "power_w_max": float(max(power)), "samples": len(sm), "reasons": sorted(reasons)}
 
@@ -357,23 +370,27 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        dl.step()
-    torch.cuda.synchronize()
-    moe.moe_profile_read()
     uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
-    barrier()
-    torch.cuda.synchronize()
     with ClockSampler(uuid) as clocks:
+        time.sleep(0.5)                      # let nvidia-smi start sampling
+        for _ in range(args.warmup):
+            dl.step()
+        torch.cuda.synchronize()
+        moe.moe_profile_read()
+        barrier()
+        torch.cuda.synchronize()
         moe.moe_profile_enable(True)
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
+        wall0 = time.time()
         ev0.record(stream)
         for _ in range(args.steps):
             dl.step()
         ev1.record(stream)
         torch.cuda.synchronize()
+        clocks.mark(wall0, time.time())
         moe.moe_profile_enable(False)
+        time.sleep(0.2)
     barrier()
     ms_total = ev0.elapsed_time(ev1)
     prof = moe.moe_profile_read()
