@@ -157,6 +157,38 @@ const char *moe_status_string(int status);
 int moe_get_device_error(void *stream);
 
 /*
+ * moe_mxfp4_forward_noalloc -- the layer of moe_mxfp4_forward_ex, for callers that
+ * cannot allocate device memory.  No counterpart in the paper.
+ *
+ * Some callers cannot call cudaMalloc or the stream-ordered allocator: a plugin
+ * handed only its input and output buffers by a host framework that owns all
+ * device memory, a serving loop that must never allocate after start-up (an
+ * allocation can block, fail under a fixed memory budget, or synchronise the
+ * device), or a process whose device memory is partitioned up front.  This call
+ * allocates nothing: its scratch is one file-scope device array of
+ * MOE_NOALLOC_SCRATCH_BYTES (32 MiB) that every GPU loading this library keeps
+ * until the process exits.
+ *   Arguments, flags and errors are those of moe_mxfp4_forward_ex without the
+ *   workspace.  Sizes whose moe_mxfp4_workspace_size exceeds
+ *   MOE_NOALLOC_SCRATCH_BYTES are refused with MOE_ERR_NO_MEMORY before anything
+ *   is enqueued (for H = I = 2880 and k = 4 that is about 364 tokens).
+ *   The first call on a device looks up the array's device address on that
+ *   device (cudaGetSymbolAddress, with the device current); make that first call
+ *   before any stream capture.  Later calls on the device reuse the address.
+ *   Every call on a device shares the one array, which keeps the previous call's
+ *   contents; the layer writes every scratch byte before it reads it, so nothing
+ *   needs clearing.  Calls whose work overlaps on the GPU (different streams
+ *   without ordering between them) race on the array: order them.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int moe_mxfp4_forward_noalloc(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E,
+                              int k, const int32_t *ids, const float *weights,
+                              const uint8_t *gate_up_blocks, const uint8_t *gate_up_scales,
+                              const float *gate_up_bias, const uint8_t *down_blocks,
+                              const uint8_t *down_scales, const float *down_bias, float alpha,
+                              float limit, uint16_t *out, uint32_t flags, void *stream);
+
+/*
  * Instrumentation (not part of the layer's math).  Kernel launches made by the
  * calls above are counted per stage; while timing is enabled each launch is also
  * bracketed by a pair of CUDA events recorded on the call's stream.

@@ -19,7 +19,10 @@ __all__ = [
     "moe_status_string", "moe_get_device_error", "MOE_FLAG_WEIGHT_ON_INPUT",
     "MOE_DEVERR_BAD_EXPERT_ID", "MOE_DEVERR_BAD_SCALE", "MOE_DEVERR_TIMEOUT",
     "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_read",
+    "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
 ]
+
+MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 MOE_FLAG_WEIGHT_ON_INPUT = 0x1
 MOE_DEVERR_BAD_EXPERT_ID = 0x1
@@ -29,7 +32,7 @@ MOE_DEVERR_TIMEOUT = 0x4
 EXPORTED_SYMBOLS = (
     "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
-    "moe_profile_enable", "moe_profile_read",
+    "moe_profile_enable", "moe_profile_read", "moe_mxfp4_forward_noalloc",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -72,6 +75,8 @@ def load_library():
     lib.moe_status_string.restype = ctypes.c_char_p
     lib.moe_get_device_error.argtypes = [p]
     lib.moe_get_device_error.restype = i32
+    lib.moe_mxfp4_forward_noalloc.argtypes = fwd + [ctypes.c_uint32, p]
+    lib.moe_mxfp4_forward_noalloc.restype = i32
     lib.moe_profile_enable.argtypes = [i32]
     lib.moe_profile_enable.restype = i32
     lib.moe_profile_read.argtypes = [p, p]
@@ -173,6 +178,19 @@ def moe_mxfp4_forward_ex(x, ids, weights, gate_up_blocks, gate_up_scales, gate_u
     nbytes = 0 if workspace is None else workspace.numel()
     rc = load_library().moe_mxfp4_forward_ex(*args, ctypes.c_uint32(flags), ws, nbytes, _stream(stream))
     _check("moe_mxfp4_forward_ex", rc)
+    return out
+
+
+def moe_mxfp4_forward_noalloc(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias,
+                              down_blocks, down_scales, down_bias, alpha: float = 1.702,
+                              limit: float = 7.0, out=None, flags: int = 0, stream=None):
+    """The layer for callers that cannot allocate device memory: the library's
+    static scratch array stands in for the workspace (see the C header for the
+    size limit, the first-call set-up and the sharing rules)."""
+    args, out = _fwd_args(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias,
+                          down_blocks, down_scales, down_bias, alpha, limit, out)
+    rc = load_library().moe_mxfp4_forward_noalloc(*args, ctypes.c_uint32(flags), _stream(stream))
+    _check("moe_mxfp4_forward_noalloc", rc)
     return out
 
 
