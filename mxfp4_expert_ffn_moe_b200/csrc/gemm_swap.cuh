@@ -1,0 +1,454 @@
+// gemm_swap.cuh -- grouped MXFP4 expert GEMM on sm_100a tensor cores, weights on
+// the MMA's M side.
+//
+// For every (expert e, token tile of up to TOK rows of that expert, 128-row weight
+// tile) of a projection:
+//   acc[n, t] = sum_k W[e, m0 + n, k] * A[row0 + t, k]          (bf16 x bf16 -> fp32)
+// with W decoded from MXFP4 (E2M1 codes, element 2j in the low nibble of byte j,
+// one E8M0 byte per 32 elements of a row) inside shared memory, then
+//   gate_up epilogue: h = acc + b_gu[e]; gate = h[2i], up = h[2i+1] (adjacent
+//                     TMEM lanes); act[row, i] = bf16(clamped SwiGLU(gate, up))
+//   down epilogue:    yp[p, n] = w[p] * (acc + b_d[e])   (router weight on output)
+//                     yp[p, n] = acc                     (router weight on input)
+// (MoE-Infinity PR #152, Changes: dequant-on-copy of fetched packed experts,
+// [N, K//2] layout, scales, bias, gate/up split, clamped SwiGLU, fp32 accumulate;
+// FreeToken PR #838: gate_up bias before the gated activation, down bias before
+// the routing weight, sum w*(y + b).)
+//
+// Why weights on M: one tcgen05.mma 128 x TOK x 16 applies every decoded weight
+// element to TOK token rows, so the in-smem decode work per MAC is 1/TOK (1/256 for
+// prefill tiles), and a tile's token count sets the MMA's N, so small decode
+// batches cost MMA time in proportion to their tokens.
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0        token TMA: per K step the token tile (32-row boxes, 128-byte
+//                 swizzle), into the ring slot the MMA freed
+//   warp 22       packed-weight TMA: per K step the weight tile (128 rows x 32 B,
+//                 3-D map, out-of-range rows zero-filled), into a deeper ring the
+//                 converters free as soon as they have read it
+//   warp 1        TMEM owner and MMA issuer (4 x 128 x N x 16 per K step)
+//   warps 2..5    epilogue (TMEM lane quarter = warp % 4)
+//   warps 6..21   converters in 4 groups; group g converts the K steps with
+//                 index % 4 == g (two 32-element blocks per thread per step)
+// Rings: token and converted-weight slots released together by the MMA; packed
+// weight slots released by the converters; two TMEM accumulators.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace swp {
+
+constexpr int BM = 128;              // weight rows per tile (TMEM lanes)
+constexpr int BK = 64;               // K elements per stage (one 128-byte swizzle row)
+constexpr int ACC_STRIDE = 256;      // TMEM columns between the two accumulators
+constexpr int TMEM_COLS = 512;
+#ifndef MOE_CONV_WARPS
+#define MOE_CONV_WARPS 16
+#endif
+#ifndef MOE_CONV_GROUPS
+#define MOE_CONV_GROUPS 4
+#endif
+constexpr int kConvWarps = MOE_CONV_WARPS;
+// Converter warps form kConvGroups groups; group g converts the K steps with
+// step index % kConvGroups == g, so that several steps (each ending in a proxy
+// fence) are converted at once.
+constexpr int kConvGroups = MOE_CONV_GROUPS;
+constexpr int kGroupThreads = 32 * kConvWarps / kConvGroups;
+constexpr int kBlocksPerThread = 2 * 128 / kGroupThreads;   // 32-element blocks per step
+constexpr int kEpiWarps = 4;
+constexpr int kWpWarp = 2 + kEpiWarps + kConvWarps;          // packed-weight TMA producer
+constexpr int kThreads = 32 * (3 + kEpiWarps + kConvWarps);
+constexpr int kFirstConvWarp = 2 + kEpiWarps;
+constexpr uint32_t WP_BYTES = BM * BK / 2;                     // 4096 packed codes
+constexpr uint32_t WB_BYTES = BM * BK * 2;                     // 16384 bf16
+constexpr uint32_t XBOX_ROWS = 32;                             // token rows per TMA box
+constexpr uint32_t XBOX_BYTES = XBOX_ROWS * BK * 2;            // 4096
+static_assert(kBlocksPerThread * kGroupThreads == BM * 2, "blocks of a step spread over a group");
+
+// Tile shapes: TOK token rows per tile; S slots of the token ring and of the
+// converted-weight ring (freed together by the MMA), PS slots of the packed-weight
+// ring (freed by the converters as soon as they have read a slot).
+template <int TOK_, int S_, int PS_>
+struct Config {
+    static constexpr int TOK = TOK_;
+    static constexpr int S = S_;
+    static constexpr int PS = PS_;
+    static constexpr uint32_t X_BYTES = TOK * BK * 2;
+    static constexpr uint32_t OFF_WB = 0;                       // S x 16 KB converted weights
+    static constexpr uint32_t OFF_X = OFF_WB + S * WB_BYTES;    // S x tokens
+    static constexpr uint32_t OFF_WP = OFF_X + S * X_BYTES;     // PS x 4 KB packed weights
+    static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES; // epilogue staging, 1 KB / warp
+    static constexpr uint32_t OFF_BAR = OFF_EPI + 1024 * kEpiWarps;
+    static constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 /*barriers*/ + 1024 /*alignment slack*/;
+    static_assert(X_BYTES % 1024 == 0, "1 KB aligned stages");
+    // a ring slot is only ever used by one converter group, so that the parity
+    // waits and the per-group arrival counts never mix two groups' steps
+    static_assert(S % kConvGroups == 0 && PS % kConvGroups == 0, "rings split over groups");
+};
+using PrefillCfg = Config<256, 4, 4>;
+using DecodeCfg = Config<32, 8, 8>;
+
+struct Params {
+    const int32_t *counts;        // [E]
+    const int32_t *offsets;       // [E + 1]
+    const int32_t *tile_offsets;  // [E + 1] in TOK-row token tiles
+    const uint8_t *wscales;       // [E, N, K/32]
+    const float *bias;            // [E, N] or null
+    int E, N, K;
+    // gate_up epilogue
+    uint16_t *act;                // [rows, N/2] bf16
+    float alpha, limit;
+    // down epilogue
+    float *yp;                    // [T*k, N] fp32, indexed by pair
+    const int32_t *sorted_pairs;  // [rows]
+    const float *weights;         // [T*k]
+    int weight_on_input;
+};
+
+__device__ __forceinline__ int tile_expert(const int32_t *__restrict__ tile_offsets, int E, int m) {
+    int lo = 0, hi = E - 1;  // largest e with tile_offsets[e] <= m
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(tile_offsets + mid) <= m)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+struct Tile {
+    int e;       // expert
+    int row0;    // first expert-ordered row (token slot) of the token tile
+    int ntok;    // token rows in the tile (1..TOK)
+    int m0;      // first weight row
+    int mrows;   // weight rows in range (64 or 128)
+};
+
+// Work item -> tile.  Items enumerate (token tile, weight tile) with the weight
+// tile fastest, so the CTAs running at one time share token tiles through L2.
+template <int TOK>
+__device__ __forceinline__ Tile decode_tile(const Params &p, int item, int w_tiles) {
+    Tile t;
+    const int g = item / w_tiles;
+    const int wt = item - g * w_tiles;
+    t.e = tile_expert(p.tile_offsets, p.E, g);
+    const int tt = g - __ldg(p.tile_offsets + t.e);
+    t.row0 = __ldg(p.offsets + t.e) + tt * TOK;
+    t.ntok = min(TOK, __ldg(p.counts + t.e) - tt * TOK);
+    t.m0 = wt * BM;
+    t.mrows = min(BM, p.N - t.m0);
+    return t;
+}
+
+// Eight E2M1 codes -> four bf16x2 words holding E2M1(code) * 2^-126 (see the
+// converter below); element order is natural (word j = elements 2j, 2j + 1).
+__device__ __forceinline__ void e2m1x8_to_bf16_rep(uint32_t q, uint32_t &r0, uint32_t &r1,
+                                                   uint32_t &r2, uint32_t &r3) {
+    const uint32_t lo = q & 0x0F0F0F0Fu;          // even elements, one per byte
+    const uint32_t hi = (q >> 4) & 0x0F0F0F0Fu;   // odd elements
+    r0 = (ptx::prmt(lo, hi, 0x8480u) * 0x1040u) & 0x81C081C0u;
+    r1 = (ptx::prmt(lo, hi, 0x8581u) * 0x1040u) & 0x81C081C0u;
+    r2 = (ptx::prmt(lo, hi, 0x8682u) * 0x1040u) & 0x81C081C0u;
+    r3 = (ptx::prmt(lo, hi, 0x8783u) * 0x1040u) & 0x81C081C0u;
+}
+
+template <class Cfg, bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_mxfp4_swap_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                              const __grid_constant__ CUtensorMap tmap_w, const Params p) {
+    constexpr int TOK = Cfg::TOK, S = Cfg::S, PS = Cfg::PS;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *const gbase = smem_raw + (base - raw);
+    auto wb_stage = [&](int c) { return base + Cfg::OFF_WB + c * WB_BYTES; };
+    auto x_stage = [&](int s) { return base + Cfg::OFF_X + s * Cfg::X_BYTES; };
+    auto wp_stage = [&](int s) { return base + Cfg::OFF_WP + s * WP_BYTES; };
+    const uint32_t bars = base + Cfg::OFF_BAR;
+    auto x_full = [&](int s) { return bars + 8u * s; };
+    auto c_full = [&](int s) { return bars + 8u * (S + s); };
+    auto empty = [&](int s) { return bars + 8u * (2 * S + s); };   // MMA done with slot s
+    auto wp_full = [&](int s) { return bars + 8u * (3 * S + s); };
+    auto wp_empty = [&](int s) { return bars + 8u * (3 * S + PS + s); };
+    auto a_full = [&](int b) { return bars + 8u * (3 * S + 2 * PS + b); };
+    auto a_empty = [&](int b) { return bars + 8u * (3 * S + 2 * PS + 2 + b); };
+    const uint32_t tmem_holder = bars + 8u * (3 * S + 2 * PS + 4);
+    static_assert(8 * (3 * S + 2 * PS + 4) + 4 <= 512, "barrier area");
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(x_full(s), 1);
+            ptx::mbar_init(c_full(s), kConvWarps / kConvGroups);
+            ptx::mbar_init(empty(s), 1);
+        }
+        for (int s = 0; s < PS; ++s) {
+            ptx::mbar_init(wp_full(s), 1);
+            ptx::mbar_init(wp_empty(s), kConvWarps / kConvGroups);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(a_full(b), 1);
+            ptx::mbar_init(a_empty(b), kEpiWarps);
+        }
+        ptx::fence_mbarrier_init();
+        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap_w);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_holder, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gbase + (tmem_holder - base));
+
+    const int w_tiles = (p.N + BM - 1) / BM;
+    const int total = __ldg(p.tile_offsets + p.E) * w_tiles;
+    const int k_iters = p.K / BK;
+    const int kblocks = p.K / 32;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ token TMA
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const Tile t = decode_tile<TOK>(p, item, w_tiles);
+                const int nbox = (t.ntok + (int)XBOX_ROWS - 1) / (int)XBOX_ROWS;
+                for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!(ok = ptx::mbar_wait(empty(s), ((it / S) & 1u) ^ 1u))) break;
+                    ptx::mbar_arrive_expect_tx(x_full(s), nbox * XBOX_BYTES);
+                    for (int b = 0; b < nbox; ++b)
+                        ptx::tma_load_2d(x_stage(s) + b * XBOX_BYTES, &tmap_x, kb * BK,
+                                         t.row0 + b * (int)XBOX_ROWS, x_full(s));
+                }
+            }
+        }
+    } else if (warp == kWpWarp) {
+        // ------------------------------------------------------------ packed-weight TMA
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const Tile t = decode_tile<TOK>(p, item, w_tiles);
+                for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                    const int s = it % PS;
+                    if (!(ok = ptx::mbar_wait(wp_empty(s), ((it / PS) & 1u) ^ 1u))) break;
+                    ptx::mbar_arrive_expect_tx(wp_full(s), WP_BYTES);
+                    ptx::tma_load_3d(wp_stage(s), &tmap_w, kb * (BK / 2), t.m0, t.e, wp_full(s));
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t it = 0, local = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
+                const Tile t = decode_tile<TOK>(p, item, w_tiles);
+                const int nmma = max(16, (t.ntok + 15) & ~15);
+                const uint32_t idesc = ptx::idesc_bf16_f32(BM, nmma);
+                const int b = local & 1;
+                if (!(ok = ptx::mbar_wait(a_empty(b), ((local >> 1) & 1u) ^ 1u))) break;
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
+                for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                    const int s = it % S;
+                    if (!(ok = ptx::mbar_wait(c_full(s), (it / S) & 1u))) break;
+                    if (!(ok = ptx::mbar_wait(x_full(s), (it / S) & 1u))) break;
+                    ptx::tc_fence_after();
+                    const uint64_t ad = ptx::sw128_kmajor_desc(wb_stage(s));
+                    const uint64_t bd = ptx::sw128_kmajor_desc(x_stage(s));
+#pragma unroll
+                    for (int j = 0; j < BK / 16; ++j)   // +32 B per 16-element K step (start address >> 4)
+                        ptx::mma_bf16(d_tmem, ad + 2u * j, bd + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
+                    ptx::mma_commit(empty(s));
+                }
+                if (ok) ptx::mma_commit(a_full(b));
+            }
+        }
+    } else if (warp < kFirstConvWarp) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                  // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;             // weight row within the tile
+        uint32_t local = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x, ++local) {
+            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const int b = local & 1;
+            if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_full(b), (local >> 1) & 1u))) break;
+            ptx::tc_fence_after();
+            const bool row_ok = r < t.mrows;
+            const int n = t.m0 + r;                             // output feature of this thread
+            const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
+            for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld_32x32b_x32(tmem_base + b * ACC_STRIDE + c0 + ((uint32_t)(q * 32) << 16), v);
+                ptx::tmem_ld_wait();
+                const int nvalid = min(32, t.ntok - c0);
+                if (kGateUp) {
+                    // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
+                    // even lane finishes tokens 0..15 of the chunk, the odd lane 16..31.
+                    // The warp's 16 features x 32 tokens go through a 1 KB staging tile
+                    // so that every lane then stores whole 16-byte pieces of act rows.
+                    const bool odd = lane & 1;
+                    const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
+                    const float bg = odd ? pb : bias, bu = odd ? bias : pb;
+                    uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + 1024 * q);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float lo_v = __uint_as_float(v[i]), hi_v = __uint_as_float(v[16 + i]);
+                        const float mine = odd ? hi_v : lo_v;
+                        const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? lo_v : hi_v, 1);
+                        const float gate = (odd ? other : mine) + bg;
+                        const float up = (odd ? mine : other) + bu;
+                        const float a = clamped_swiglu(gate, up, p.alpha, p.limit);
+                        stg[(odd ? 16 + i : i) * 16 + (lane >> 1)] = (uint16_t)(pack_bf16x2(a, 0.0f) & 0xFFFFu);
+                    }
+                    __syncwarp();
+                    const int64_t fbase = (t.m0 + 32 * q) >> 1;     // first feature of the warp
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int piece = lane + 32 * h;            // 64 pieces of 16 bytes
+                        const int tok = piece >> 1;
+                        if (tok < nvalid) {
+                            const uint4 val = *reinterpret_cast<const uint4 *>(stg + tok * 16 + (piece & 1) * 8);
+                            *reinterpret_cast<uint4 *>(p.act + (int64_t)(t.row0 + c0 + tok) * (p.N / 2) +
+                                                       fbase + (piece & 1) * 8) = val;
+                        }
+                    }
+                    __syncwarp();
+                } else {
+                    int pair = 0;
+                    float wgt = 1.0f;
+                    if (lane < nvalid) {
+                        pair = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
+                        if (!p.weight_on_input) wgt = __ldg(p.weights + pair);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int pi = __shfl_sync(0xFFFFFFFFu, pair, i);
+                        const float wi = __shfl_sync(0xFFFFFFFFu, wgt, i);
+                        if (row_ok && i < nvalid)
+                            p.yp[(int64_t)pi * p.N + n] = wi * (__uint_as_float(v[i]) + bias);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(a_empty(b));
+        }
+    } else {
+        // ------------------------------------------------------------ converters
+        // Each thread turns kBlocksPerThread 32-element blocks (16 bytes of codes
+        // each) of the step's weight rows into bf16: the codes become E2M1 * 2^-126
+        // bit patterns (sign to bit 15, exponent bits and mantissa msb to bits 8..6;
+        // code 1 = 0.5 is the bf16 subnormal 2^-127), then one bf16 multiply by
+        // 2^(s-1) (two, by 2^126 and 2^(s-127), when 2^(s-1) is not a bf16) gives
+        // E2M1 * 2^(s-127) exactly; the result goes to the 128-byte swizzled
+        // K-major layout the MMA reads.  The E8M0 bytes a thread needs for its
+        // group's next step are loaded from global memory one step ahead.
+        const int ct = threadIdx.x - 32 * kFirstConvWarp;
+        const int grp = ct / kGroupThreads;
+        const int gt = ct % kGroupThreads;                    // thread within its group
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const uint8_t *srow[kBlocksPerThread];
+            bool rok[kBlocksPerThread];
+#pragma unroll
+            for (int bi = 0; bi < kBlocksPerThread; ++bi) {
+                const int blkid = gt + bi * kGroupThreads;
+                const int row = blkid >> 1;
+                rok[bi] = row < t.mrows;
+                srow[bi] = p.wscales + ((int64_t)t.e * p.N + t.m0 + (rok[bi] ? row : 0)) * kblocks + (blkid & 1);
+            }
+            // first step of this tile that belongs to this group
+            int kb = (int)((grp - (int)(it % kConvGroups) + kConvGroups) % kConvGroups);
+            uint32_t nxt[kBlocksPerThread];
+#pragma unroll
+            for (int bi = 0; bi < kBlocksPerThread; ++bi)
+                nxt[bi] = (rok[bi] && kb < k_iters) ? (uint32_t)__ldg(srow[bi] + 2 * kb) : 127u;
+            for (; kb < k_iters; kb += kConvGroups) {
+                const uint32_t gi = it + (uint32_t)kb;         // global step index
+                const int c = gi % S, ps = gi % PS;
+                uint32_t cur[kBlocksPerThread];
+#pragma unroll
+                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
+                    cur[bi] = nxt[bi];
+                    nxt[bi] = (rok[bi] && kb + kConvGroups < k_iters)
+                                  ? (uint32_t)__ldg(srow[bi] + 2 * (kb + kConvGroups)) : 127u;
+                }
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (gi / PS) & 1u)))) break;
+                uint4 q4[kBlocksPerThread];
+#pragma unroll
+                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
+                    const int blkid = gt + bi * kGroupThreads;
+                    q4[bi] = ptx::ld_shared_v4(wp_stage(ps) + (blkid >> 1) * 32 + (blkid & 1) * 16);
+                }
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(c), ((gi / S) & 1u) ^ 1u)))) break;
+#pragma unroll
+                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
+                    const int blkid = gt + bi * kGroupThreads;    // 0 .. 255 within the step
+                    const int row = blkid >> 1, blk = blkid & 1;
+                    const uint32_t sc = cur[bi];
+                    uint32_t m1, m2 = 0;
+                    if (sc == 255u) {
+                        raise_device_error(MOE_DEVERR_BAD_SCALE);
+                        m1 = 0x7FC07FC0u;
+                    } else if (sc <= 128u) {
+                        m1 = ((sc + 126u) << 7) * 0x10001u;
+                    } else {
+                        m1 = 0x7E807E80u;
+                        m2 = (sc << 7) * 0x10001u;
+                    }
+                    const uint32_t qw[4] = {q4[bi].x, q4[bi].y, q4[bi].z, q4[bi].w};
+                    const uint32_t dst_row = wb_stage(c) + row * 128;
+                    const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t r0, r1, r2, r3;
+                        e2m1x8_to_bf16_rep(qw[w], r0, r1, r2, r3);
+                        r0 = ptx::hmul2_bf16(r0, m1);
+                        r1 = ptx::hmul2_bf16(r1, m1);
+                        r2 = ptx::hmul2_bf16(r2, m1);
+                        r3 = ptx::hmul2_bf16(r3, m1);
+                        if (m2) {
+                            r0 = ptx::hmul2_bf16(r0, m2);
+                            r1 = ptx::hmul2_bf16(r1, m2);
+                            r2 = ptx::hmul2_bf16(r2, m2);
+                            r3 = ptx::hmul2_bf16(r3, m2);
+                        }
+                        const uint32_t chunk = (uint32_t)(blk * 4 + w);
+                        ptx::st_shared_v4(dst_row + ((chunk ^ sw) << 4), r0, r1, r2, r3);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(c_full(c));
+                    // every lane has consumed its packed words (the conversion used
+                    // them), so the TMA may refill the packed slot
+                    ptx::mbar_arrive(wp_empty(ps));
+                }
+            }
+            it += (uint32_t)k_iters;
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace swp
+}  // namespace moe

@@ -16,7 +16,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
-#include "gemm_tc.cuh"
+#include "gemm_swap.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -117,45 +117,50 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// bf16 activations [rows, K], K-major: box of 64 elements (128 B, swizzled) x BM rows.
+// bf16 activations [rows, K], K-major: box of 64 elements (128 B, swizzled) x 32 rows.
 bool make_act_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t K) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
-    cuuint32_t box[2] = {(cuuint32_t)moe::tc::BK, (cuuint32_t)moe::tc::BM};
+    cuuint32_t box[2] = {(cuuint32_t)moe::swp::BK, moe::swp::XBOX_ROWS};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// packed MXFP4 codes [E, N, K/2] bytes: box of 32 bytes (64 codes) x BN rows x 1 expert.
+// packed MXFP4 codes [E, N, K/2] bytes: box of 32 bytes (64 codes) x 128 rows x 1 expert.
 bool make_weight_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
     cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
-    cuuint32_t box[3] = {(cuuint32_t)(moe::tc::BK / 2), (cuuint32_t)moe::tc::BN, 1};
+    cuuint32_t box[3] = {(cuuint32_t)(moe::swp::BK / 2), (cuuint32_t)moe::swp::BM, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kGateUp>
+int max_smem_optin() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+    return v;
+}
+
+// Grouped projection: rows of A (expert order, [rows, K] bf16) x packed weights
+// [E, N, K/2] of each row's expert, with the gate_up or the down epilogue.
+template <class Cfg, bool kGateUp>
 int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, const uint8_t *wblocks,
                         const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
                         const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
                         uint16_t *act, float alpha, float limit, float *yp,
                         const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
-    CUtensorMap ma, mw;
-    if (!make_act_map(&ma, A, rows, K) || !make_weight_map(&mw, wblocks, E, N, K)) return MOE_ERR_CUDA;
-    if (cudaFuncSetAttribute(moe::tc::grouped_mxfp4_tc_kernel<kGateUp>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)moe::tc::SMEM_BYTES) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    moe::tc::Params p{};
+    CUtensorMap mx, mw;
+    if (!make_act_map(&mx, A, rows, K) || !make_weight_map(&mw, wblocks, E, N, K)) return MOE_ERR_CUDA;
+    moe::swp::Params p{};
     p.counts = counts;
     p.offsets = offsets;
     p.tile_offsets = tile_offsets;
@@ -171,14 +176,41 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     p.sorted_pairs = sorted_pairs;
     p.weights = weights;
     p.weight_on_input = woi;
-    const int64_t n_tiles = moe::ceil_div(N, moe::tc::BN);
-    const int64_t max_tiles = (moe::ceil_div(rows, moe::tc::BM) + E) * n_tiles;
-    const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
+    const uint32_t smem = Cfg::SMEM_BYTES;
+    if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
+    auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int64_t w_tiles = moe::ceil_div(N, moe::swp::BM);
+    const int64_t max_items = (moe::ceil_div(rows, Cfg::TOK) + E) * w_tiles;
+    const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
     StageScope scope(stage, s);
-    moe::tc::grouped_mxfp4_tc_kernel<kGateUp>
-        <<<grid, moe::tc::kThreads, moe::tc::SMEM_BYTES, s>>>(ma, mw, p);
+    kernel<<<grid, moe::swp::kThreads, smem, s>>>(mx, mw, p);
     return launch_check();
 }
+
+// Both projections with one tile configuration.
+template <class Cfg>
+int launch_projections(const uint16_t *x_perm, uint16_t *act, float *yp, int64_t P, int64_t H,
+                       int64_t I, int64_t E, const uint8_t *gate_up_blocks,
+                       const uint8_t *gate_up_scales, const float *gate_up_bias,
+                       const uint8_t *down_blocks, const uint8_t *down_scales,
+                       const float *down_bias, float alpha, float limit, const int32_t *counts,
+                       const int32_t *offsets, const int32_t *tile_offsets,
+                       const int32_t *sorted_pairs, const float *weights, bool woi, cudaStream_t s) {
+    int rc = launch_grouped_gemm<Cfg, true>(MOE_STAGE_GATE_UP, x_perm, P, H, gate_up_blocks,
+                                            gate_up_scales, gate_up_bias, E, 2 * I, counts, offsets,
+                                            tile_offsets, act, alpha, limit, nullptr, sorted_pairs,
+                                            weights, 0, s);
+    if (rc != MOE_OK) return rc;
+    return launch_grouped_gemm<Cfg, false>(MOE_STAGE_DOWN, act, P, I, down_blocks, down_scales,
+                                           down_bias, E, H, counts, offsets, tile_offsets, nullptr,
+                                           alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
+}
+
+// Token tiles of 32 rows (deep weight pipeline) when experts see few rows on
+// average, 256-row tiles otherwise.
+bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
 
 }  // namespace
 
@@ -260,7 +292,8 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
     const bool woi = (flags & MOE_FLAG_WEIGHT_ON_INPUT) != 0;
     if (woi && (gate_up_bias || down_bias)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gate_up_blocks, 16) ||
-        !aligned(down_blocks, 16) || !aligned(ids, 4) || !aligned(weights, 4) ||
+        !aligned(down_blocks, 16) || !aligned(gate_up_scales, 16) || !aligned(down_scales, 16) ||
+        !aligned(ids, 4) || !aligned(weights, 4) ||
         !aligned(gate_up_bias, 4) || !aligned(down_bias, 4))
         return MOE_ERR_INVALID_ARG;
     if (workspace && !aligned(workspace, kAlign)) return MOE_ERR_INVALID_ARG;
@@ -287,13 +320,15 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
     float *yp = reinterpret_cast<float *>(ws + L.yp);
 
     const int64_t P = T * k;
+    const bool decode_tiles = use_decode_tiles(P, E);
     int rc = MOE_OK;
     do {
         {
             const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
             StageScope sp(MOE_STAGE_PERMUTE, s);
             moe::permute_pairs_kernel<<<1, moe::kPermuteThreads, perm_smem, s>>>(
-                ids, P, (int)E, moe::tc::BM, counts, offsets, tile_offsets, sorted_pairs);
+                ids, P, (int)E, decode_tiles ? moe::swp::DecodeCfg::TOK : moe::swp::PrefillCfg::TOK, counts,
+                offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
         {
@@ -303,16 +338,16 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                 x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
         }
         if ((rc = launch_check()) != MOE_OK) break;
-        if ((rc = launch_grouped_gemm<true>(MOE_STAGE_GATE_UP, x_perm, P, H, gate_up_blocks,
-                                            gate_up_scales, gate_up_bias, E, 2 * I, counts, offsets,
-                                            tile_offsets, act, alpha, limit, nullptr, sorted_pairs,
-                                            weights, 0, s)) != MOE_OK)
-            break;
-        if ((rc = launch_grouped_gemm<false>(MOE_STAGE_DOWN, act, P, I, down_blocks, down_scales,
-                                             down_bias, E, H, counts, offsets, tile_offsets, nullptr,
-                                             alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0,
-                                             s)) != MOE_OK)
-            break;
+        rc = decode_tiles
+                 ? launch_projections<moe::swp::DecodeCfg>(
+                       x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias,
+                       down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,
+                       tile_offsets, sorted_pairs, weights, woi, s)
+                 : launch_projections<moe::swp::PrefillCfg>(
+                       x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias,
+                       down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,
+                       tile_offsets, sorted_pairs, weights, woi, s);
+        if (rc != MOE_OK) break;
         {
             const int64_t n4 = T * (H / 4);
             const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;

@@ -36,11 +36,29 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
         : "memory");
 }
 
+// One potentially blocking test of the phase: the hardware may suspend the
+// thread for up to `kSuspendNs` waiting for the phase to complete, so waiting
+// warps sleep instead of taking issue slots from the working ones.
+constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per try
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of the phase (cheap when the phase has already completed).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -48,28 +66,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Wait until the phase of parity `parity` has completed.  Gives up after about
-// four seconds of wall time (far beyond any legitimate wait of this pipeline),
-// raising MOE_DEVERR_TIMEOUT and returning false so that the caller can wind down
-// instead of keeping the GPU busy forever.
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+// Wait until the phase of parity `parity` has completed.  Bounded: after tries
+// adding up to about four seconds (far beyond any legitimate wait of this
+// pipeline) it raises MOE_DEVERR_TIMEOUT and returns false so that the caller
+// can wind down instead of keeping the GPU busy forever.  The cycle counter is a
+// second bound in case a try returns early without the phase having completed.
+constexpr long long kWaitLimitCycles = 8000000000ll;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
+    const long long t0 = clock64();
+#pragma unroll 1
+    for (uint32_t i = 1; i < 4000u; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-            raise_device_error(MOE_DEVERR_TIMEOUT);
-            return false;
-        }
+        if (clock64() - t0 > kWaitLimitCycles) break;
     }
+    raise_device_error(MOE_DEVERR_TIMEOUT);
+    return false;
+}
+
+// Named CTA barrier `id` (1..15) over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---- TMA --------------------------------------------------------------------
@@ -90,6 +109,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, 
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// Contiguous global -> shared copy by the TMA engine (16-byte aligned addresses,
+// size a multiple of 16), completing on `bar` with `bytes` transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
         : "memory");
 }
 
