@@ -80,8 +80,8 @@ struct Config {
     static constexpr uint32_t OFF_WB = 0;                       // S x 16 KB converted weights
     static constexpr uint32_t OFF_X = OFF_WB + S * WB_BYTES;    // S x tokens
     static constexpr uint32_t OFF_WP = OFF_X + S * X_BYTES;     // PS x 4 KB packed weights
-    static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES; // epilogue staging, 1 KB / warp
-    static constexpr uint32_t OFF_BAR = OFF_EPI + 1024 * kEpiWarps;
+    static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES; // epilogue staging, 4 KB / warp
+    static constexpr uint32_t OFF_BAR = OFF_EPI + 4096 * kEpiWarps;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 /*barriers*/ + 1024 /*alignment slack*/;
     static_assert(X_BYTES % 1024 == 0, "1 KB aligned stages");
     // a ring slot is only ever used by one converter group, so that the parity
@@ -169,21 +169,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto x_stage = [&](int s) { return base + Cfg::OFF_X + s * Cfg::X_BYTES; };
     auto wp_stage = [&](int s) { return base + Cfg::OFF_WP + s * WP_BYTES; };
     const uint32_t bars = base + Cfg::OFF_BAR;
-    auto x_full = [&](int s) { return bars + 8u * s; };
-    auto c_full = [&](int s) { return bars + 8u * (S + s); };
+    // ready(s): the token tile landed (producer arrival + transaction bytes) and
+    // every converter warp of the step's group stored its weights
+    auto ready = [&](int s) { return bars + 8u * s; };
     auto empty = [&](int s) { return bars + 8u * (2 * S + s); };   // MMA done with slot s
     auto wp_full = [&](int s) { return bars + 8u * (3 * S + s); };
     auto wp_empty = [&](int s) { return bars + 8u * (3 * S + PS + s); };
     auto a_full = [&](int b) { return bars + 8u * (3 * S + 2 * PS + b); };
     auto a_empty = [&](int b) { return bars + 8u * (3 * S + 2 * PS + 2 + b); };
     const uint32_t tmem_holder = bars + 8u * (3 * S + 2 * PS + 4);
-    static_assert(8 * (3 * S + 2 * PS + 4) + 4 <= 512, "barrier area");
+    static_assert(8 * (3 * S + 2 * PS + 4) + 4 <= 512, "barrier area");   // (slots S..2S-1 unused)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(x_full(s), 1);
-            ptx::mbar_init(c_full(s), kConvWarps / kConvGroups);
+            ptx::mbar_init(ready(s), 1 + kConvWarps / kConvGroups);
             ptx::mbar_init(empty(s), 1);
         }
         for (int s = 0; s < PS; ++s) {
@@ -214,64 +214,70 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ token TMA
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const Tile t = decode_tile<TOK>(p, item, w_tiles);
-                const int nbox = (t.ntok + (int)XBOX_ROWS - 1) / (int)XBOX_ROWS;
-                for (int kb = 0; kb < k_iters; ++kb, ++it) {
-                    const int s = it % S;
-                    if (!(ok = ptx::mbar_wait(empty(s), ((it / S) & 1u) ^ 1u))) break;
-                    ptx::mbar_arrive_expect_tx(x_full(s), nbox * XBOX_BYTES);
+        // The whole warp runs the loop (uniform control flow keeps the operands in
+        // uniform registers); one elected lane issues the asynchronous copies.
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const int nbox = (t.ntok + (int)XBOX_ROWS - 1) / (int)XBOX_ROWS;
+            for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                const int s = it % S;
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(s), ((it / S) & 1u) ^ 1u)))) break;
+                if (ptx::elect_one()) {
+                    ptx::mbar_arrive_expect_tx(ready(s), nbox * XBOX_BYTES);
                     for (int b = 0; b < nbox; ++b)
                         ptx::tma_load_2d(x_stage(s) + b * XBOX_BYTES, &tmap_x, kb * BK,
-                                         t.row0 + b * (int)XBOX_ROWS, x_full(s));
+                                         t.row0 + b * (int)XBOX_ROWS, ready(s));
                 }
+                __syncwarp();
             }
         }
     } else if (warp == kWpWarp) {
         // ------------------------------------------------------------ packed-weight TMA
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const Tile t = decode_tile<TOK>(p, item, w_tiles);
-                for (int kb = 0; kb < k_iters; ++kb, ++it) {
-                    const int s = it % PS;
-                    if (!(ok = ptx::mbar_wait(wp_empty(s), ((it / PS) & 1u) ^ 1u))) break;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                const int s = it % PS;
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_empty(s), ((it / PS) & 1u) ^ 1u)))) break;
+                if (ptx::elect_one()) {
                     ptx::mbar_arrive_expect_tx(wp_full(s), WP_BYTES);
                     ptx::tma_load_3d(wp_stage(s), &tmap_w, kb * (BK / 2), t.m0, t.e, wp_full(s));
                 }
+                __syncwarp();
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t it = 0, local = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-                const Tile t = decode_tile<TOK>(p, item, w_tiles);
-                const int nmma = max(16, (t.ntok + 15) & ~15);
-                const uint32_t idesc = ptx::idesc_bf16_f32(BM, nmma);
-                const int b = local & 1;
-                if (!(ok = ptx::mbar_wait(a_empty(b), ((local >> 1) & 1u) ^ 1u))) break;
+        // Warp-wide loop, one elected lane issues the MMAs and commits.
+        uint32_t it = 0, local = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
+            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const int nmma = max(16, (t.ntok + 15) & ~15);
+            const uint32_t idesc = ptx::idesc_bf16_f32(BM, nmma);
+            const int b = local & 1;
+            if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_empty(b), ((local >> 1) & 1u) ^ 1u)))) break;
+            ptx::tc_fence_after();
+            const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
+            for (int kb = 0; kb < k_iters; ++kb, ++it) {
+                const int s = it % S;
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(ready(s), (it / S) & 1u)))) break;
                 ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem_base + b * ACC_STRIDE;
-                for (int kb = 0; kb < k_iters; ++kb, ++it) {
-                    const int s = it % S;
-                    if (!(ok = ptx::mbar_wait(c_full(s), (it / S) & 1u))) break;
-                    if (!(ok = ptx::mbar_wait(x_full(s), (it / S) & 1u))) break;
-                    ptx::tc_fence_after();
-                    const uint64_t ad = ptx::sw128_kmajor_desc(wb_stage(s));
-                    const uint64_t bd = ptx::sw128_kmajor_desc(x_stage(s));
+                const uint64_t ad = ptx::sw128_kmajor_desc(wb_stage(s));
+                const uint64_t bd = ptx::sw128_kmajor_desc(x_stage(s));
+                if (ptx::elect_one()) {
 #pragma unroll
                     for (int j = 0; j < BK / 16; ++j)   // +32 B per 16-element K step (start address >> 4)
                         ptx::mma_bf16(d_tmem, ad + 2u * j, bd + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
                     ptx::mma_commit(empty(s));
                 }
-                if (ok) ptx::mma_commit(a_full(b));
+                __syncwarp();
             }
+            if (ok && ptx::elect_one()) ptx::mma_commit(a_full(b));
+            __syncwarp();
         }
     } else if (warp < kFirstConvWarp) {
         // ------------------------------------------------------------ epilogue
@@ -286,6 +292,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = r < t.mrows;
             const int n = t.m0 + r;                             // output feature of this thread
             const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
+            // down: lane i holds the pair index and routing weight of token 32 j + i
+            int pairs[TOK / 32];
+            float wts[TOK / 32];
+            if (!kGateUp) {
+#pragma unroll
+                for (int j = 0; j < TOK / 32; ++j) {
+                    const int tok = 32 * j + lane;
+                    pairs[j] = tok < t.ntok ? __ldg(p.sorted_pairs + t.row0 + tok) : 0;
+                    wts[j] = (tok < t.ntok && !p.weight_on_input) ? __ldg(p.weights + pairs[j]) : 1.0f;
+                }
+            }
             for (int c0 = 0; c0 < t.ntok; c0 += 32) {
                 uint32_t v[32];
                 ptx::tmem_ld_32x32b_x32(tmem_base + b * ACC_STRIDE + c0 + ((uint32_t)(q * 32) << 16), v);
@@ -299,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool odd = lane & 1;
                     const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
                     const float bg = odd ? pb : bias, bu = odd ? bias : pb;
-                    uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + 1024 * q);
+                    uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + 4096 * q);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const float lo_v = __uint_as_float(v[i]), hi_v = __uint_as_float(v[16 + i]);
@@ -324,19 +341,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     __syncwarp();
                 } else {
-                    int pair = 0;
-                    float wgt = 1.0f;
-                    if (lane < nvalid) {
-                        pair = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
-                        if (!p.weight_on_input) wgt = __ldg(p.weights + pair);
-                    }
+                    // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
+                    // so that each pair's row segment leaves as 16-byte stores
+                    float *stg = reinterpret_cast<float *>(gbase + Cfg::OFF_EPI + 4096 * q);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int pi = __shfl_sync(0xFFFFFFFFu, pair, i);
-                        const float wi = __shfl_sync(0xFFFFFFFFu, wgt, i);
-                        if (row_ok && i < nvalid)
-                            p.yp[(int64_t)pi * p.N + n] = wi * (__uint_as_float(v[i]) + bias);
+                        const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], i);
+                        stg[i * 32 + lane] = wi * (__uint_as_float(v[i]) + bias);
                     }
+                    __syncwarp();
+                    if (32 * q < t.mrows) {                      // warp-uniform
+#pragma unroll
+                        for (int rd = 0; rd < 8; ++rd) {
+                            const int piece = rd * 32 + lane;    // 32 tokens x 8 pieces of 16 B
+                            const int tok = piece >> 3, part = piece & 7;
+                            const int pi = __shfl_sync(0xFFFFFFFFu, pairs[c0 >> 5], tok);
+                            if (tok < nvalid) {
+                                const float4 val = *reinterpret_cast<const float4 *>(stg + tok * 32 + part * 4);
+                                *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
+                            }
+                        }
+                    }
+                    __syncwarp();
                 }
             }
             ptx::tc_fence_before();
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    ptx::mbar_arrive(c_full(c));
+                    ptx::mbar_arrive(ready(c));
                     // every lane has consumed its packed words (the conversion used
                     // them), so the TMA may refill the packed slot
                     ptx::mbar_arrive(wp_empty(ps));
