@@ -176,7 +176,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     p.sorted_pairs = sorted_pairs;
     p.weights = weights;
     p.weight_on_input = woi;
-    const uint32_t smem = Cfg::SMEM_BYTES;
+    const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
     auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -211,6 +211,39 @@ int launch_projections(const uint16_t *x_perm, uint16_t *act, float *yp, int64_t
 // Token tiles of 32 rows (deep weight pipeline) when experts see few rows on
 // average, 256-row tiles otherwise.
 bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
+
+#ifndef MOE_DECODE_A_TMEM
+#define MOE_DECODE_A_TMEM 1
+#endif
+#ifndef MOE_PREFILL_A_TMEM
+#define MOE_PREFILL_A_TMEM 0
+#endif
+
+// Tile configurations of the grouped GEMMs.  The TMEM-operand variants hold two
+// tiles' scale rows (128 x K/32 bytes each) in shared memory; for K too large for
+// that they give way to the shared-memory-operand variant of the same tiles.
+enum TileConfig { kDecodeSmem, kDecodeTmem, kPrefillSmem, kPrefillTmem };
+
+template <class Cfg>
+bool config_fits(int64_t H, int64_t I) {
+    const int optin = max_smem_optin();
+    return (int)Cfg::smem_bytes((int)(H / 32)) <= optin && (int)Cfg::smem_bytes((int)(I / 32)) <= optin;
+}
+
+TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E) {
+    if (use_decode_tiles(P, E))
+        return (MOE_DECODE_A_TMEM && config_fits<moe::swp::DecodeTmemCfg>(H, I)) ? kDecodeTmem : kDecodeSmem;
+    return (MOE_PREFILL_A_TMEM && config_fits<moe::swp::PrefillTmemCfg>(H, I)) ? kPrefillTmem : kPrefillSmem;
+}
+
+int config_tok(TileConfig c) {
+    switch (c) {
+        case kDecodeSmem: return moe::swp::DecodeCfg::TOK;
+        case kDecodeTmem: return moe::swp::DecodeTmemCfg::TOK;
+        case kPrefillSmem: return moe::swp::PrefillCfg::TOK;
+        default: return moe::swp::PrefillTmemCfg::TOK;
+    }
+}
 
 }  // namespace
 
@@ -320,14 +353,14 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
     float *yp = reinterpret_cast<float *>(ws + L.yp);
 
     const int64_t P = T * k;
-    const bool decode_tiles = use_decode_tiles(P, E);
+    const TileConfig cfg = pick_config(P, H, I, E);
     int rc = MOE_OK;
     do {
         {
             const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
             StageScope sp(MOE_STAGE_PERMUTE, s);
             moe::permute_pairs_kernel<<<1, moe::kPermuteThreads, perm_smem, s>>>(
-                ids, P, (int)E, decode_tiles ? moe::swp::DecodeCfg::TOK : moe::swp::PrefillCfg::TOK, counts,
+                ids, P, (int)E, config_tok(cfg), counts,
                 offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
@@ -338,15 +371,17 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                 x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
         }
         if ((rc = launch_check()) != MOE_OK) break;
-        rc = decode_tiles
-                 ? launch_projections<moe::swp::DecodeCfg>(
-                       x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias,
-                       down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,
-                       tile_offsets, sorted_pairs, weights, woi, s)
-                 : launch_projections<moe::swp::PrefillCfg>(
-                       x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias,
-                       down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,
-                       tile_offsets, sorted_pairs, weights, woi, s);
+#define MOE_PROJECTIONS(C)                                                                       \
+    launch_projections<C>(x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias, \
+                          down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,         \
+                          tile_offsets, sorted_pairs, weights, woi, s)
+        switch (cfg) {
+            case kDecodeSmem: rc = MOE_PROJECTIONS(moe::swp::DecodeCfg); break;
+            case kDecodeTmem: rc = MOE_PROJECTIONS(moe::swp::DecodeTmemCfg); break;
+            case kPrefillSmem: rc = MOE_PROJECTIONS(moe::swp::PrefillCfg); break;
+            default: rc = MOE_PROJECTIONS(moe::swp::PrefillTmemCfg); break;
+        }
+#undef MOE_PROJECTIONS
         if (rc != MOE_OK) break;
         {
             const int64_t n4 = T * (H / 4);
