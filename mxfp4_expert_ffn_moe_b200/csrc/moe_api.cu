@@ -16,8 +16,10 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
+#include "gemm_mxf.cuh"
 #include "gemm_swap.cuh"
 #include "permute.cuh"
+#include "split.cuh"
 #include "route.cuh"
 
 namespace {
@@ -30,6 +32,8 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace carve-up; offsets in bytes from the workspace base.
 struct Workspace {
+    // x_perm / act: bf16 rows, or (block-scaled path) the rows split into two E4M3
+    // planes with per-step scale slots
     size_t counts, offsets, tile_offsets, sorted_pairs, x_perm, act, yp, total;
 };
 
@@ -46,8 +50,12 @@ Workspace workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int k) {
     w.offsets = take(sizeof(int32_t) * (E + 1));
     w.tile_offsets = take(sizeof(int32_t) * (E + 1));
     w.sorted_pairs = take(sizeof(int32_t) * P);
-    w.x_perm = take(sizeof(uint16_t) * P * H);
-    w.act = take(sizeof(uint16_t) * P * I);
+    const auto rows_bytes = [&](int64_t K) {
+        const int64_t bf16 = int64_t(sizeof(uint16_t)) * P * K, split = 2 * P * moe::split_row_bytes(K);
+        return (size_t)(bf16 > split ? bf16 : split);
+    };
+    w.x_perm = take(rows_bytes(H));
+    w.act = take(rows_bytes(I));
     w.yp = take(sizeof(float) * P * H);
     w.total = off;
     return w;
@@ -143,6 +151,49 @@ bool make_weight_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int6
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// split activations [2][rows][K] bytes (hi plane, lo plane): box of 128 bytes
+// (swizzled) x 16 rows x 1 plane.
+bool make_split_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int64_t RS = moe::split_row_bytes(K);
+    cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, 2};
+    cuuint64_t strides[2] = {(cuuint64_t)RS, (cuuint64_t)(rows * RS)};
+    cuuint32_t box[3] = {(cuuint32_t)moe::mxf::BK, (cuuint32_t)moe::mxf::XBOX_ROWS, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the 16-byte per-step scale slots of the same rows: box of 16 bytes x 16 rows x 1 plane.
+bool make_split_scale_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int64_t RS = moe::split_row_bytes(K);
+    cuuint64_t dims[3] = {(cuuint64_t)(RS - K), (cuuint64_t)rows, 2};
+    cuuint64_t strides[2] = {(cuuint64_t)RS, (cuuint64_t)(rows * RS)};
+    cuuint32_t box[3] = {16, (cuuint32_t)moe::mxf::XBOX_ROWS, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(ptr + K), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// packed MXFP4 codes [E, N, K/2] bytes: box of 128 bytes (256 codes, 128-byte
+// swizzle) x 128 rows x 1 expert.
+bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
+    cuuint32_t box[3] = {moe::mxf::WP_ROW, (cuuint32_t)moe::mxf::BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int max_smem_optin() {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -208,6 +259,75 @@ int launch_projections(const uint16_t *x_perm, uint16_t *act, float *yp, int64_t
                                            alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
 }
 
+// Block-scaled grouped projection: split rows B ([2][P][K] + scale words) x packed
+// weights [E, N, K/2] of each row's expert, with the gate_up or the down epilogue.
+template <class Cfg, bool kGateUp>
+int launch_mxf_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const uint8_t *wblocks,
+                    const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
+                    const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
+                    uint8_t *actq, float alpha, float limit, float *yp,
+                    const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
+    CUtensorMap mb, mbs, mw;
+    if (!make_split_map(&mb, bq, P, K) || !make_split_scale_map(&mbs, bq, P, K) ||
+        !make_packed_map(&mw, wblocks, E, N, K))
+        return MOE_ERR_CUDA;
+    moe::mxf::Params p{};
+    p.counts = counts;
+    p.offsets = offsets;
+    p.tile_offsets = tile_offsets;
+    p.wscales = wscales;
+    p.bias = bias;
+    p.E = (int)E;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.P = (int)P;
+    p.actq = actq;
+    p.alpha = alpha;
+    p.limit = limit;
+    p.yp = yp;
+    p.sorted_pairs = sorted_pairs;
+    p.weights = weights;
+    p.weight_on_input = woi;
+    const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
+    if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
+    auto kernel = moe::mxf::grouped_mxfp4_mxf_kernel<Cfg, kGateUp>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int64_t w_tiles = moe::ceil_div(N, moe::mxf::BM);
+    const int64_t max_items = (moe::ceil_div(P, Cfg::TOK) + E) * w_tiles;
+    const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
+    StageScope scope(stage, s);
+    kernel<<<grid, Cfg::kThreads, smem, s>>>(mb, mbs, mw, p);
+    return launch_check();
+}
+
+// Split of the gathered rows, then both projections on the block-scaled path.
+template <class Cfg>
+int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sorted_pairs,
+                     uint8_t *xq, uint8_t *actq, float *yp, int64_t P,
+                     int64_t H, int64_t I, int64_t E, int k, const uint8_t *gate_up_blocks,
+                     const uint8_t *gate_up_scales, const float *gate_up_bias,
+                     const uint8_t *down_blocks, const uint8_t *down_scales,
+                     const float *down_bias, float alpha, float limit, const int32_t *counts,
+                     const int32_t *offsets, const int32_t *tile_offsets, bool woi, cudaStream_t s) {
+    {
+        const int64_t items = P * moe::ceil_div(H, 128);
+        const int64_t grid = moe::ceil_div(items, 8) < sm_count() * 8 ? moe::ceil_div(items, 8) : sm_count() * 8;
+        StageScope sg(MOE_STAGE_GATHER, s);
+        moe::split_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(x, weights, sorted_pairs, offsets, (int)E, k,
+                                                               H, P, woi ? 1 : 0, xq);
+    }
+    int rc = launch_check();
+    if (rc != MOE_OK) return rc;
+    rc = launch_mxf_gemm<Cfg, true>(MOE_STAGE_GATE_UP, xq, P, H, gate_up_blocks, gate_up_scales,
+                                    gate_up_bias, E, 2 * I, counts, offsets, tile_offsets, actq,
+                                    alpha, limit, nullptr, sorted_pairs, weights, 0, s);
+    if (rc != MOE_OK) return rc;
+    return launch_mxf_gemm<Cfg, false>(MOE_STAGE_DOWN, actq, P, I, down_blocks, down_scales,
+                                       down_bias, E, H, counts, offsets, tile_offsets, nullptr,
+                                       alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
+}
+
 // Token tiles of 32 rows (deep weight pipeline) when experts see few rows on
 // average, 256-row tiles otherwise.
 bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
@@ -222,7 +342,14 @@ bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
 // Tile configurations of the grouped GEMMs.  The TMEM-operand variants hold two
 // tiles' scale rows (128 x K/32 bytes each) in shared memory; for K too large for
 // that they give way to the shared-memory-operand variant of the same tiles.
-enum TileConfig { kDecodeSmem, kDecodeTmem, kPrefillSmem, kPrefillTmem };
+enum TileConfig { kDecodeSmem, kDecodeTmem, kPrefillSmem, kPrefillTmem, kDecodeMxf, kPrefillMxf };
+
+#ifndef MOE_MXF_DECODE
+#define MOE_MXF_DECODE 1
+#endif
+#ifndef MOE_MXF_PREFILL
+#define MOE_MXF_PREFILL 0
+#endif
 
 template <class Cfg>
 bool config_fits(int64_t H, int64_t I) {
@@ -231,6 +358,8 @@ bool config_fits(int64_t H, int64_t I) {
 }
 
 TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E) {
+    if (use_decode_tiles(P, E) && MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) return kDecodeMxf;
+    if (!use_decode_tiles(P, E) && MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) return kPrefillMxf;
     if (use_decode_tiles(P, E))
         return (MOE_DECODE_A_TMEM && config_fits<moe::swp::DecodeTmemCfg>(H, I)) ? kDecodeTmem : kDecodeSmem;
     return (MOE_PREFILL_A_TMEM && config_fits<moe::swp::PrefillTmemCfg>(H, I)) ? kPrefillTmem : kPrefillSmem;
@@ -241,6 +370,8 @@ int config_tok(TileConfig c) {
         case kDecodeSmem: return moe::swp::DecodeCfg::TOK;
         case kDecodeTmem: return moe::swp::DecodeTmemCfg::TOK;
         case kPrefillSmem: return moe::swp::PrefillCfg::TOK;
+        case kDecodeMxf: return moe::mxf::DecodeCfg::TOK;
+        case kPrefillMxf: return moe::mxf::PrefillCfg::TOK;
         default: return moe::swp::PrefillTmemCfg::TOK;
     }
 }
@@ -364,24 +495,38 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                 offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
-        {
-            const int64_t gather_grid = moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
-            StageScope sg(MOE_STAGE_GATHER, s);
-            moe::gather_rows_kernel<<<(unsigned)gather_grid, 256, 0, s>>>(
-                x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
-        }
-        if ((rc = launch_check()) != MOE_OK) break;
+        const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
+        if (mxf) {
+            uint8_t *xq = reinterpret_cast<uint8_t *>(x_perm);
+            uint8_t *actq = reinterpret_cast<uint8_t *>(act);
+#define MOE_MXF_LAYER(C)                                                                          \
+    launch_mxf_layer<C>(x, weights, sorted_pairs, xq, actq, yp, P, H, I, E, k, gate_up_blocks,           \
+                        gate_up_scales, gate_up_bias, down_blocks, down_scales, down_bias, alpha,    \
+                        limit, counts, offsets, tile_offsets, woi, s)
+            rc = cfg == kDecodeMxf ? MOE_MXF_LAYER(moe::mxf::DecodeCfg) : MOE_MXF_LAYER(moe::mxf::PrefillCfg);
+#undef MOE_MXF_LAYER
+            if (rc != MOE_OK) break;
+        } else {
+            {
+                const int64_t gather_grid =
+                    moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
+                StageScope sg(MOE_STAGE_GATHER, s);
+                moe::gather_rows_kernel<<<(unsigned)gather_grid, 256, 0, s>>>(
+                    x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
+            }
+            if ((rc = launch_check()) != MOE_OK) break;
 #define MOE_PROJECTIONS(C)                                                                       \
     launch_projections<C>(x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias, \
                           down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,         \
                           tile_offsets, sorted_pairs, weights, woi, s)
-        switch (cfg) {
-            case kDecodeSmem: rc = MOE_PROJECTIONS(moe::swp::DecodeCfg); break;
-            case kDecodeTmem: rc = MOE_PROJECTIONS(moe::swp::DecodeTmemCfg); break;
-            case kPrefillSmem: rc = MOE_PROJECTIONS(moe::swp::PrefillCfg); break;
-            default: rc = MOE_PROJECTIONS(moe::swp::PrefillTmemCfg); break;
-        }
+            switch (cfg) {
+                case kDecodeSmem: rc = MOE_PROJECTIONS(moe::swp::DecodeCfg); break;
+                case kDecodeTmem: rc = MOE_PROJECTIONS(moe::swp::DecodeTmemCfg); break;
+                case kPrefillSmem: rc = MOE_PROJECTIONS(moe::swp::PrefillCfg); break;
+                default: rc = MOE_PROJECTIONS(moe::swp::PrefillTmemCfg); break;
+            }
 #undef MOE_PROJECTIONS
+        }
         if (rc != MOE_OK) break;
         {
             const int64_t n4 = T * (H / 4);
