@@ -62,8 +62,9 @@ constexpr int XBOX_ROWS = 16;                    // token rows per TMA box
 constexpr uint32_t XBOX_BYTES = XBOX_ROWS * BK;  // one E4M3 term of 16 rows
 constexpr int kEpiWarps = 4;
 constexpr int kFirstStageWarp = 2 + kEpiWarps;
-constexpr uint32_t kEpiStage = 4096;             // staging bytes per epilogue warp
+constexpr uint32_t kEpiStage = 2048;             // staging bytes per epilogue warp
 constexpr uint32_t kXchBytes = 2 * 4 * 32 * 4;   // per-token block maxima exchanged by warp pairs
+constexpr uint32_t kSinkBytes = 128;             // scratch words (see ptx::sink_shared)
 
 // TOK token rows per tile (B has 2 TOK rows: hi and lo terms); S slots of the
 // unpacked-weight / token / scale-factor rings (freed together by the MMA); PS slots
@@ -93,12 +94,21 @@ struct Config {
     static constexpr uint32_t OFF_WP = OFF_X + S * X_BYTES;
     static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES;
     static constexpr uint32_t OFF_XCH = OFF_EPI + kEpiStage * kEpiWarps;
-    static constexpr uint32_t OFF_BAR = OFF_XCH + kXchBytes;
+    static constexpr uint32_t OFF_SINK = OFF_XCH + kXchBytes;
+    static constexpr uint32_t OFF_BAR = OFF_SINK + kSinkBytes;
     static constexpr uint32_t BAR_BYTES = 8 * (3 * S + 2 * PS + 2 * NACC + 6) + 16;
     static constexpr uint32_t OFF_SC = (OFF_BAR + BAR_BYTES + 127u) & ~127u;
     static constexpr uint32_t SMEM_FIXED = OFF_SC + 1024;   // + slack for the 1 KB base alignment
     static_assert(TOK % 32 == 0 && TOK <= 128, "token tile: B rows <= 256");
     static_assert(S % G == 0, "a ring slot belongs to one stager group");
+    // A stager group may only wait on a packed slot whose previous load it also read
+    // (an mbarrier parity wait cannot tell a phase from the one two phases later), so
+    // the set of groups reading a packed slot must not change from load to load: the
+    // groups read consecutive loads in a fixed rotation of G / WP_STEPS loads, and
+    // tiles run a multiple of KALIGN steps.
+    static_assert(G <= WP_STEPS ? WP_STEPS % G == 0 : (G % WP_STEPS == 0 && PS % (G / WP_STEPS) == 0),
+                  "packed slots read by a fixed set of stager groups");
+    static constexpr int KALIGN = G > WP_STEPS ? G : WP_STEPS;
     static_assert(NACC == 1 || NACC == 2, "one or two accumulators");
     static_assert(TMEM_USED <= 512, "TMEM columns");
     static_assert(X_BYTES % 1024 == 0 && WP_BYTES % 1024 == 0, "1 KB aligned stages");
@@ -255,8 +265,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 
     const int w_tiles = (p.N + BM - 1) / BM;
     const int total = __ldg(p.tile_offsets + p.E) * w_tiles;
-    const int k_iters = (p.K + BK - 1) / BK;
-    const int wp_loads = (k_iters + WP_STEPS - 1) / WP_STEPS;   // packed loads per tile
+    // K steps per tile, rounded up to KALIGN: the extra steps read only the TMA's zero
+    // fill (codes and token rows past K) with scale 1 and add nothing
+    const int k_iters = ((p.K + BK - 1) / BK + Cfg::KALIGN - 1) / Cfg::KALIGN * Cfg::KALIGN;
+    const int wp_loads = k_iters / WP_STEPS;   // packed loads per tile
 
     if (warp == 0) {
         // ------------------------------------------------------------ token TMA
@@ -358,13 +370,22 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
             const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
             const uint32_t acc = tmem_base + b * Cfg::ACC_COLS + lane_off;
             for (int c0 = 0; c0 < t.ntok; c0 += 32, ++chunk) {
-                uint32_t vh[32], vl[32];
+                // hi-term columns, then the lo-term columns added in two pieces of 16
+                // (keeps the live registers at 48)
+                uint32_t vh[32];
                 ptx::tmem_ld_32x32b_x32(acc + c0, vh);
-                ptx::tmem_ld_32x32b_x32(acc + t.h + c0, vl);
                 ptx::tmem_ld_wait();
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vh[i]) + __uint_as_float(vl[i]);
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vh[i]);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t vl[16];
+                    ptx::tmem_ld_32x32b_x16(acc + t.h + c0 + 16 * hf, vl);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[16 * hf + i] += __uint_as_float(vl[i]);
+                }
                 const int nvalid = min(32, t.ntok - c0);
                 if (kGateUp) {
                     // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
@@ -438,26 +459,30 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                         pair_l = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
                         if (!p.weight_on_input) wt_l = __ldg(p.weights + pair_l);
                     }
+                    // two passes of 16 tokens through a 2 KB staging tile
                     float *stg = reinterpret_cast<float *>(gbase + Cfg::OFF_EPI + kEpiStage * q);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float wi = __shfl_sync(0xFFFFFFFFu, wt_l, i);
-                        stg[i * 32 + lane] = wi * (v[i] + bias);
-                    }
-                    __syncwarp();
-                    if (32 * q < t.mrows) {                      // warp-uniform
+                    for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-                        for (int rd = 0; rd < 8; ++rd) {
-                            const int piece = rd * 32 + lane;    // 32 tokens x 8 pieces of 16 B
-                            const int tok = piece >> 3, part = piece & 7;
-                            const int pi = __shfl_sync(0xFFFFFFFFu, pair_l, tok);
-                            if (tok < nvalid) {
-                                const float4 val = *reinterpret_cast<const float4 *>(stg + tok * 32 + part * 4);
-                                *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
+                        for (int i = 0; i < 16; ++i) {
+                            const float wi = __shfl_sync(0xFFFFFFFFu, wt_l, 16 * hf + i);
+                            stg[i * 32 + lane] = wi * (v[16 * hf + i] + bias);
+                        }
+                        __syncwarp();
+                        if (32 * q < t.mrows) {                  // warp-uniform
+#pragma unroll
+                            for (int rd = 0; rd < 4; ++rd) {
+                                const int piece = rd * 32 + lane;    // 16 tokens x 8 pieces of 16 B
+                                const int tok = 16 * hf + (piece >> 3), part = piece & 7;
+                                const int pi = __shfl_sync(0xFFFFFFFFu, pair_l, tok);
+                                if (tok < nvalid) {
+                                    const float4 val = *reinterpret_cast<const float4 *>(stg + (piece >> 3) * 32 + part * 4);
+                                    *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
+                                }
                             }
                         }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
             }
             ptx::tc_fence_before();
@@ -496,7 +521,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                 for (int c = 0; c < 4; ++c) {
                     const int rw = lane + 32 * c;
                     uint32_t w = 0x7F7F7F7Fu;
-                    if (rw < t.mrows) {
+                    if (rw < t.mrows && kb0 < kblocks) {
                         const uint32_t a = scb + (uint32_t)(rw * kblocks + kb0);
                         const uint32_t lo16 = ptx::ld_shared_u16(a);
                         const uint32_t hi16 = (kb0 + 2 < kblocks) ? ptx::ld_shared_u16(a + 2) : 0x7F7Fu;
@@ -513,7 +538,13 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                 const uint32_t src = wp_stage(ps) + row * WP_ROW;
                 const uint32_t c0 = 4u * (uint32_t)(kb % WP_STEPS), sw = (uint32_t)(row & 7);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pk[i] = ptx::ld_shared_v4(src + (((c0 + (uint32_t)i) ^ sw) << 4));
+                for (int i = 0; i < 4; ++i) pk[i] = ptx::ld_volatile_shared_v4(src + (((c0 + (uint32_t)i) ^ sw) << 4));
+                // hand the packed slot back to the TMA at once, after every lane's four
+                // loads have landed (volatile loads are never repeated after this)
+                ptx::sink_shared(base + Cfg::OFF_SINK + 4u * (uint32_t)(warp & 31),
+                                 pk[0].x ^ pk[1].x ^ pk[2].x ^ pk[3].x);
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(wp_empty(ps));
                 // the slot is free (MMA done) and the token rows with their scale slots landed
                 if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(s), ((gi / S) & 1u) ^ 1u) &&
                                                         ptx::mbar_wait(b_full(s), (gi / S) & 1u))))
@@ -551,12 +582,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(ready(s));
-                    ptx::mbar_arrive(wp_empty(ps));
-                    // a tile's last load may hold a single step: arrive for the missing one
-                    if (kb % WP_STEPS == 0 && kb + 1 >= k_iters) ptx::mbar_arrive(wp_empty(ps));
-                }
+                if (lane == 0) ptx::mbar_arrive(ready(s));
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(sc_empty(sb));
@@ -579,10 +605,16 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 #define MOE_MXF_DECODE_PS 4
 #endif
 #ifndef MOE_MXF_DECODE_G
-#define MOE_MXF_DECODE_G 2
+#define MOE_MXF_DECODE_G 4
 #endif
 using DecodeCfg = Config<32, MOE_MXF_DECODE_S, MOE_MXF_DECODE_PS, 2, MOE_MXF_DECODE_G>;
-using PrefillCfg = Config<128, 2, 2, 1, 1>;
+#ifndef MOE_MXF_PREFILL_S
+#define MOE_MXF_PREFILL_S 3
+#endif
+#ifndef MOE_MXF_PREFILL_G
+#define MOE_MXF_PREFILL_G 1
+#endif
+using PrefillCfg = Config<128, MOE_MXF_PREFILL_S, 2, 1, MOE_MXF_PREFILL_G>;
 
 }  // namespace mxf
 }  // namespace moe
