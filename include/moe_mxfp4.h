@@ -171,7 +171,7 @@ int moe_get_device_error(void *stream);
  *   Arguments, flags and errors are those of moe_mxfp4_forward_ex without the
  *   workspace.  Sizes whose moe_mxfp4_workspace_size exceeds
  *   MOE_NOALLOC_SCRATCH_BYTES are refused with MOE_ERR_NO_MEMORY before anything
- *   is enqueued (for H = I = 2880 and k = 4 that is about 364 tokens).
+ *   is enqueued (for H = I = 2880 and k = 4 that is about 340 tokens).
  *   The first call on a device looks up the array's device address on that
  *   device (cudaGetSymbolAddress, with the device current); make that first call
  *   before any stream capture.  Later calls on the device reuse the address.
