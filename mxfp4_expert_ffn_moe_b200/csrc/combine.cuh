@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const float *__restri
                                                            const int32_t *__restrict__ ids,
                                                            int64_t T, int k, int E, int64_t H,
                                                            uint16_t *__restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t q = H / 4;
     const int64_t n = T * q;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;

@@ -48,4 +48,14 @@ __device__ __forceinline__ float clamped_swiglu(float gate, float up, float alph
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch.  pdl_wait(): block until the preceding kernel of
+// the stream has completed and its writes are visible (returns at once when this
+// kernel was launched without the programmatic-serialisation attribute); every
+// kernel of the layer calls it before its first read of data a predecessor writes
+// and before its first global write.  pdl_trigger(): let the next kernel of the
+// stream be scheduled now (its blocks start as resources free up and then wait in
+// their own pdl_wait), hiding launch latency and prologues.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace moe

@@ -261,6 +261,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
+    // barriers and TMEM are set up; wait for the producer of this kernel's inputs
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gbase + (tmem_holder - base));
 
     const int w_tiles = (p.N + BM - 1) / BM;

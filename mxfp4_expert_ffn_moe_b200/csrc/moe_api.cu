@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
 #include <vector>
 
 #include <cuda.h>
@@ -70,6 +71,24 @@ bool forward_sizes_ok(int64_t T, int64_t H, int64_t I, int64_t E, int k) {
 }
 
 int launch_check() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled while
+// its predecessor in the stream is still running; every kernel of the layer calls
+// pdl_wait() before touching data its predecessor writes (see common.cuh).
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);   // errors surface in launch_check
+}
 
 // ---- per-stage launch counting and optional CUDA-event timing ---------------
 struct TimedLaunch {
@@ -236,7 +255,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     const int64_t max_items = (moe::ceil_div(rows, Cfg::TOK) + E) * w_tiles;
     const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
     StageScope scope(stage, s);
-    kernel<<<grid, moe::swp::kThreads, smem, s>>>(mx, mw, p);
+    launch_pdl(kernel, dim3(grid), dim3(moe::swp::kThreads), smem, s, mx, mw, p);
     return launch_check();
 }
 
@@ -297,7 +316,7 @@ int launch_mxf_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const ui
     const int64_t max_items = (moe::ceil_div(P, Cfg::TOK) + E) * w_tiles;
     const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
     StageScope scope(stage, s);
-    kernel<<<grid, Cfg::kThreads, smem, s>>>(mb, mbs, mw, p);
+    launch_pdl(kernel, dim3(grid), dim3(Cfg::kThreads), smem, s, mb, mbs, mw, p);
     return launch_check();
 }
 
@@ -314,8 +333,8 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
         const int64_t items = P * moe::ceil_div(H, 128);
         const int64_t grid = moe::ceil_div(items, 8) < sm_count() * 8 ? moe::ceil_div(items, 8) : sm_count() * 8;
         StageScope sg(MOE_STAGE_GATHER, s);
-        moe::split_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(x, weights, sorted_pairs, offsets, (int)E, k,
-                                                               H, P, woi ? 1 : 0, xq);
+        launch_pdl(moe::split_rows_kernel, dim3((unsigned)grid), dim3(256), 0, s, x, weights, sorted_pairs,
+                   offsets, (int)E, k, H, P, woi ? 1 : 0, xq);
     }
     int rc = launch_check();
     if (rc != MOE_OK) return rc;
@@ -490,9 +509,8 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
         {
             const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
             StageScope sp(MOE_STAGE_PERMUTE, s);
-            moe::permute_pairs_kernel<<<1, moe::kPermuteThreads, perm_smem, s>>>(
-                ids, P, (int)E, config_tok(cfg), counts,
-                offsets, tile_offsets, sorted_pairs);
+            launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P,
+                       (int)E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
         const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
@@ -511,8 +529,8 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                 const int64_t gather_grid =
                     moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
                 StageScope sg(MOE_STAGE_GATHER, s);
-                moe::gather_rows_kernel<<<(unsigned)gather_grid, 256, 0, s>>>(
-                    x, weights, sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
+                launch_pdl(moe::gather_rows_kernel, dim3((unsigned)gather_grid), dim3(256), 0, s, x, weights,
+                           sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
             }
             if ((rc = launch_check()) != MOE_OK) break;
 #define MOE_PROJECTIONS(C)                                                                       \
@@ -532,7 +550,8 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
             const int64_t n4 = T * (H / 4);
             const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;
             StageScope sc(MOE_STAGE_COMBINE, s);
-            moe::combine_rows_kernel<<<(unsigned)cgrid, 256, 0, s>>>(yp, ids, T, k, (int)E, H, out);
+            launch_pdl(moe::combine_rows_kernel, dim3((unsigned)cgrid), dim3(256), 0, s, yp, ids, T, k, (int)E, H,
+                       out);
         }
         rc = launch_check();
     } while (0);

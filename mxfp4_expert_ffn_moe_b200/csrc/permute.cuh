@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     const int32_t *__restrict__ ids, int64_t P, int E, int bm, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
     int32_t *__restrict__ sorted_pairs) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int sm_perm[];
     int *cnt = sm_perm;             // [32][E]: per-warp counts, then per-warp running bases
     int *off = sm_perm + 32 * E;    // [E + 1]: expert start rows
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
     const uint16_t *__restrict__ x, const float *__restrict__ weights,
     const int32_t *__restrict__ sorted_pairs, const int32_t *__restrict__ offsets, int E, int k,
     int64_t H, int weight_on_input, uint16_t *__restrict__ x_perm) {
+    pdl_wait();
+    pdl_trigger();
     const int rows = offsets[E];
     const int lane = threadIdx.x & 31;
     const int wpb = blockDim.x >> 5;
@@ -103,15 +107,23 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
         const float w = weight_on_input ? weights[p] : 1.0f;
-        for (int64_t c = lane; c < chunks; c += 32) {
-            uint4 v = __ldg(src + c);
-            if (weight_on_input) {
-                v.x = pack_bf16x2(bf16lo_to_f32(v.x) * w, bf16hi_to_f32(v.x) * w);
-                v.y = pack_bf16x2(bf16lo_to_f32(v.y) * w, bf16hi_to_f32(v.y) * w);
-                v.z = pack_bf16x2(bf16lo_to_f32(v.z) * w, bf16hi_to_f32(v.z) * w);
-                v.w = pack_bf16x2(bf16lo_to_f32(v.w) * w, bf16hi_to_f32(v.w) * w);
+        // four 16-byte loads in flight per lane before their stores
+        for (int64_t c0 = lane; c0 < chunks; c0 += 4 * 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c0 + 32 * u < chunks) v[u] = __ldg(src + c0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (c0 + 32 * u >= chunks) continue;
+                if (weight_on_input) {
+                    v[u].x = pack_bf16x2(bf16lo_to_f32(v[u].x) * w, bf16hi_to_f32(v[u].x) * w);
+                    v[u].y = pack_bf16x2(bf16lo_to_f32(v[u].y) * w, bf16hi_to_f32(v[u].y) * w);
+                    v[u].z = pack_bf16x2(bf16lo_to_f32(v[u].z) * w, bf16hi_to_f32(v[u].z) * w);
+                    v[u].w = pack_bf16x2(bf16lo_to_f32(v[u].w) * w, bf16hi_to_f32(v[u].w) * w);
+                }
+                dst[c0 + 32 * u] = v[u];
             }
-            dst[c] = v;
         }
     }
 }

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
     const uint16_t *__restrict__ x, const float *__restrict__ weights,
     const int32_t *__restrict__ sorted_pairs, const int32_t *__restrict__ offsets, int E, int k,
     int64_t K, int64_t P, int weight_on_input, uint8_t *__restrict__ xq) {
+    pdl_wait();
+    pdl_trigger();
     const int rows = offsets[E];
     const int lane = threadIdx.x & 31;
     const int64_t steps = (K + 127) / 128;
