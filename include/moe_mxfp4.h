@@ -192,7 +192,16 @@ int moe_mxfp4_forward_noalloc(const uint16_t *x, int64_t T, int64_t H, int64_t I
  * Instrumentation (not part of the layer's math).  Kernel launches made by the
  * calls above are counted per stage; while timing is enabled each launch is also
  * bracketed by a pair of CUDA events recorded on the call's stream.
- *   moe_profile_enable(on)        on != 0 starts event timing, 0 stops it.
+ *   moe_profile_enable(on)        on != 0 starts event timing of every stage, 0
+ *                                 stops it.
+ *   moe_profile_enable_stages(mask) times only the stages whose bit (1 << stage)
+ *                                 is set (0 stops timing); bits past
+ *                                 MOE_PROFILE_STAGES give MOE_ERR_INVALID_ARG.
+ *                                 An event pair sits between a stage's kernel and
+ *                                 its neighbours in the stream, so timing a stage
+ *                                 keeps that kernel from overlapping their tails
+ *                                 (programmatic dependent launch); untimed
+ *                                 stages keep it.
  *   moe_profile_read(ms, launches) waits for every recorded event, writes the
  *                                 summed kernel milliseconds and the launch counts
  *                                 per stage (arrays of MOE_PROFILE_STAGES entries,
@@ -211,6 +220,7 @@ enum {
     MOE_STAGE_DEQUANT = 6  /* mxfp4_dequantize                            */
 };
 int moe_profile_enable(int on);
+int moe_profile_enable_stages(uint32_t stage_mask);
 int moe_profile_read(double *ms, int64_t *launches);
 
 #ifdef __cplusplus

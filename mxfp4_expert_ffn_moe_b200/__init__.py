@@ -18,7 +18,8 @@ __all__ = [
     "moe_mxfp4_forward", "moe_mxfp4_forward_ex", "moe_mxfp4_workspace_size",
     "moe_status_string", "moe_get_device_error", "MOE_FLAG_WEIGHT_ON_INPUT",
     "MOE_DEVERR_BAD_EXPERT_ID", "MOE_DEVERR_BAD_SCALE", "MOE_DEVERR_TIMEOUT",
-    "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_read",
+    "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_enable_stages",
+    "moe_profile_read",
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -32,7 +33,7 @@ MOE_DEVERR_TIMEOUT = 0x4
 EXPORTED_SYMBOLS = (
     "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
-    "moe_profile_enable", "moe_profile_read", "moe_mxfp4_forward_noalloc",
+    "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -79,6 +80,8 @@ def load_library():
     lib.moe_mxfp4_forward_noalloc.restype = i32
     lib.moe_profile_enable.argtypes = [i32]
     lib.moe_profile_enable.restype = i32
+    lib.moe_profile_enable_stages.argtypes = [ctypes.c_uint32]
+    lib.moe_profile_enable_stages.restype = i32
     lib.moe_profile_read.argtypes = [p, p]
     lib.moe_profile_read.restype = i32
     _lib = lib
@@ -209,6 +212,14 @@ def moe_get_device_error(stream=None) -> int:
 def moe_profile_enable(on: bool = True) -> None:
     """Start (or stop) CUDA-event timing of every kernel the library launches."""
     _check("moe_profile_enable", load_library().moe_profile_enable(1 if on else 0))
+
+
+def moe_profile_enable_stages(stages) -> None:
+    """Time only the named stages (an iterable of PROFILE_STAGES names); empty stops."""
+    mask = 0
+    for name in stages:
+        mask |= 1 << PROFILE_STAGES.index(name)
+    _check("moe_profile_enable_stages", load_library().moe_profile_enable_stages(ctypes.c_uint32(mask)))
 
 
 def moe_profile_read():

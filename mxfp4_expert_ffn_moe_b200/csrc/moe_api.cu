@@ -96,7 +96,7 @@ struct TimedLaunch {
     cudaEvent_t start, stop;
 };
 struct Profiler {
-    bool timing = false;
+    uint32_t timed_stages = 0;   // bit i: bracket stage i's launches with events
     int64_t launches[MOE_PROFILE_STAGES] = {};
     std::vector<TimedLaunch> pending;
 };
@@ -107,7 +107,8 @@ class StageScope {
    public:
     StageScope(int stage, cudaStream_t s) : stage_(stage), s_(s) {
         ++g_prof.launches[stage];
-        if (g_prof.timing && cudaEventCreate(&a_) == cudaSuccess && cudaEventCreate(&b_) == cudaSuccess)
+        if (((g_prof.timed_stages >> stage) & 1u) && cudaEventCreate(&a_) == cudaSuccess &&
+            cudaEventCreate(&b_) == cudaSuccess)
             cudaEventRecord(a_, s_);
         else
             a_ = b_ = nullptr;
@@ -572,7 +573,13 @@ int moe_mxfp4_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_
 }
 
 int moe_profile_enable(int on) {
-    g_prof.timing = on != 0;
+    g_prof.timed_stages = on ? (1u << MOE_PROFILE_STAGES) - 1u : 0u;
+    return MOE_OK;
+}
+
+int moe_profile_enable_stages(uint32_t stage_mask) {
+    if (stage_mask >> MOE_PROFILE_STAGES) return MOE_ERR_INVALID_ARG;
+    g_prof.timed_stages = stage_mask;
     return MOE_OK;
 }
 
