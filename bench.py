@@ -30,6 +30,10 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 
 DEFAULT_WORKLOAD = "20b_prefill_T4096"
+# DRAM bytes (read + write) of one gate_up launch of the default workload, from the ncu
+# capture summarised in profiles/traffic_grouped_mxfp4_swap_kernel_20b_prefill.md; valid
+# for that kernel build only (set to None when the kernel changes until re-captured)
+GATE_UP_DRAM_BYTES = 462.85e6
 METRIC = "MoE layer tokens/s (prefill)"
 # algorithmic weight bytes of one gpt-oss-20b/120b expert (gate_up + down: packed
 # codes, E8M0 scales, fp32 biases)
@@ -468,7 +472,7 @@ def run_ours(args):
     long_region = ms_total > 1000.0
     peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": "gate_up grouped GEMM",
+                "frac": achieved / peak, "traffic": GATE_UP_DRAM_BYTES, "kernel": "gate_up grouped GEMM",
                 "peak_kind": f"{peaks['source']} bf16 {'sustained' if long_region else 'burst'}",
                 "frac_of_2250_spec": achieved / 2250.0,
                 "flops_per_launch": gu_flops, "avg_launch_ms": gu_avg}

@@ -54,9 +54,16 @@ namespace mxf {
 constexpr int BM = 128;                          // weight rows per tile (TMEM lanes)
 constexpr int BK = 128;                          // K elements per step
 constexpr int KBS = BK / 32;                     // scale blocks per step
-constexpr int WP_STEPS = 2;                      // K steps per packed-weight load
-constexpr uint32_t WP_ROW = WP_STEPS * BK / 2;   // 128 packed bytes per weight row and load
-constexpr uint32_t WP_BYTES = BM * WP_ROW;       // packed codes of a load (128-byte swizzle)
+#ifndef MOE_MXF_WP_STEPS
+#define MOE_MXF_WP_STEPS 2
+#endif
+// K steps per packed-weight load: 2 (128-byte rows, 128-byte swizzle) or 4 (256-byte
+// rows, unswizzled; stagers read a row's chunks in a lane-rotated order)
+constexpr int WP_STEPS = MOE_MXF_WP_STEPS;
+static_assert(WP_STEPS == 2 || WP_STEPS == 4, "two or four K steps per packed load");
+constexpr uint32_t WP_ROW = WP_STEPS * BK / 2;   // packed bytes per weight row and load
+constexpr bool WP_SWIZZLED = WP_ROW == 128;
+constexpr uint32_t WP_BYTES = BM * WP_ROW;       // packed codes of a load
 constexpr uint32_t WA_BYTES = BM * BK;           // unpacked codes of a step
 constexpr int XBOX_ROWS = 16;                    // token rows per TMA box
 constexpr uint32_t XBOX_BYTES = XBOX_ROWS * BK;  // one E4M3 term of 16 rows
@@ -537,11 +544,19 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                 if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (pj / PS) & 1u)))) break;
                 // this step's 64 bytes: 16-byte chunks 4 (kb % 2) .. + 3 of the row's
                 // swizzled 128-byte line
+                // the step's 64 bytes are 16-byte chunks c0 .. c0 + 3 of the row's line; load i
+                // fetches logical chunk lc[i] (128-byte rows: swizzled positions; 256-byte rows:
+                // chunks taken in a lane-rotated order so a warp's loads spread over banks)
                 uint4 pk[4];
+                uint32_t lc[4];
                 const uint32_t src = wp_stage(ps) + row * WP_ROW;
                 const uint32_t c0 = 4u * (uint32_t)(kb % WP_STEPS), sw = (uint32_t)(row & 7);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pk[i] = ptx::ld_volatile_shared_v4(src + (((c0 + (uint32_t)i) ^ sw) << 4));
+                for (int i = 0; i < 4; ++i) {
+                    lc[i] = WP_SWIZZLED ? (uint32_t)i : (uint32_t)((i + row) & 3);
+                    const uint32_t phys = WP_SWIZZLED ? ((c0 + lc[i]) ^ sw) : (c0 + lc[i]);
+                    pk[i] = ptx::ld_volatile_shared_v4(src + (phys << 4));
+                }
                 // hand the packed slot back to the TMA at once, after every lane's four
                 // loads have landed (volatile loads are never repeated after this)
                 ptx::sink_shared(base + Cfg::OFF_SINK + 4u * (uint32_t)(warp & 31),
@@ -568,8 +583,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                 const uint32_t sw128 = (uint32_t)(row & 7);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    ptx::st_shared_v4(dst + (((uint32_t)(2 * i) ^ sw128) << 4), pk[i].x, pk[i].y, 0u, 0u);
-                    ptx::st_shared_v4(dst + (((uint32_t)(2 * i + 1) ^ sw128) << 4), pk[i].z, pk[i].w, 0u, 0u);
+                    ptx::st_shared_v4(dst + (((2u * lc[i]) ^ sw128) << 4), pk[i].x, pk[i].y, 0u, 0u);
+                    ptx::st_shared_v4(dst + (((2u * lc[i] + 1u) ^ sw128) << 4), pk[i].z, pk[i].w, 0u, 0u);
                 }
                 const uint32_t sf = tmem_base + lane_off + Cfg::SF_COL0 + s * Cfg::SF_STRIDE;
                 ptx::tmem_st_32x32b_x4(sf, sfa);
@@ -610,7 +625,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
 #ifndef MOE_MXF_DECODE_G
 #define MOE_MXF_DECODE_G 4
 #endif
-using DecodeCfg = Config<32, MOE_MXF_DECODE_S, MOE_MXF_DECODE_PS, 2, MOE_MXF_DECODE_G>;
+using DecodeCfg = Config<32, MOE_MXF_DECODE_S, MOE_MXF_DECODE_PS * 2 / WP_STEPS, 2, MOE_MXF_DECODE_G>;
 #ifndef MOE_MXF_PREFILL_S
 #define MOE_MXF_PREFILL_S 3
 #endif

@@ -200,8 +200,8 @@ bool make_split_scale_map(CUtensorMap *m, const uint8_t *ptr, int64_t rows, int6
                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// packed MXFP4 codes [E, N, K/2] bytes: box of 128 bytes (256 codes, 128-byte
-// swizzle) x 128 rows x 1 expert.
+// packed MXFP4 codes [E, N, K/2] bytes: box of WP_ROW bytes (128: 128-byte swizzle;
+// 256: unswizzled) x 128 rows x 1 expert.
 bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -210,7 +210,8 @@ bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int6
     cuuint32_t box[3] = {moe::mxf::WP_ROW, (cuuint32_t)moe::mxf::BM, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE,
+               moe::mxf::WP_SWIZZLED ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -85,3 +85,17 @@ def test_argument_checks_need_no_device(lib):
     # a caller workspace that is too small is refused before anything runs
     assert lib.moe_mxfp4_forward_ex(*args, ctypes.c_uint32(0), ctypes.c_void_p(0x100000), 64,
                                     null) == -4
+
+
+def test_profiler_stage_mask_host_logic(lib):
+    # host-side state only: no event is recorded while no launch happens
+    assert lib.moe_profile_enable_stages(ctypes.c_uint32(1 << 7)) == -1        # past the stages
+    assert lib.moe_profile_enable_stages(ctypes.c_uint32(1 << 3)) == 0         # gate_up only
+    moe.moe_profile_enable_stages(["gate_up", "down"])
+    moe.moe_profile_enable_stages([])
+    moe.moe_profile_enable(False)
+    ms = (ctypes.c_double * 7)()
+    launches = (ctypes.c_int64 * 7)()
+    assert lib.moe_profile_read(ms, launches) == 0
+    with pytest.raises(ValueError):
+        moe.moe_profile_enable_stages(["no_such_stage"])
