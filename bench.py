@@ -33,7 +33,7 @@ DEFAULT_WORKLOAD = "20b_prefill_T4096"
 # DRAM bytes (read + write) of one gate_up launch of the default workload, from the ncu
 # capture summarised in profiles/traffic_grouped_mxfp4_swap_kernel_20b_prefill.md; valid
 # for that kernel build only (set to None when the kernel changes until re-captured)
-GATE_UP_DRAM_BYTES = 462.85e6
+GATE_UP_DRAM_BYTES = 458.48e6
 METRIC = "MoE layer tokens/s (prefill)"
 # algorithmic weight bytes of one gpt-oss-20b/120b expert (gate_up + down: packed
 # codes, E8M0 scales, fp32 biases)

@@ -69,71 +69,35 @@ static_assert(kBlocksPerThread * kGroupThreads == BM * 2, "blocks of a step spre
 
 // Tile shapes: TOK token rows per tile; S slots of the token ring and of the
 // converted-weight ring (freed together by the MMA), PS slots of the packed-weight
-// ring (freed by the converters as soon as they have read a slot).
-//
-// A_TMEM selects where the converted weights (the MMA's A operand) live:
-//   false: S x 16 KB swizzled bf16 tiles in shared memory (smem descriptor)
-//   true:  S x 32 columns of tensor memory next to the accumulators; each
-//          converter thread writes its weight row's 64 bf16 values of a step with
-//          one tcgen05.st, which keeps 32 KB per step of converter stores and MMA
-//          operand reads off shared memory.  The E8M0 bytes of a weight tile then
-//          arrive with one bulk copy per tile (the tile's rows are contiguous in
-//          [E, N, K/32]) into a two-slot ring placed after the barriers.
-// NACC accumulators of max(TOK, 32) fp32 columns each (two let the epilogue of one
-// tile overlap the MMAs of the next).
-template <int TOK_, int S_, int PS_, bool A_TMEM_ = false, int NACC_ = 2>
+// ring (freed by the converters as soon as they have read a slot).  Two TMEM
+// accumulators of max(TOK, 32) fp32 columns each let the epilogue of one tile
+// overlap the MMAs of the next.
+template <int TOK_, int S_, int PS_>
 struct Config {
     static constexpr int TOK = TOK_;
     static constexpr int S = S_;
     static constexpr int PS = PS_;
-    static constexpr bool A_TMEM = A_TMEM_;
-    static constexpr int NACC = NACC_;
+    static constexpr int NACC = 2;
     static constexpr uint32_t ACC_STRIDE = TOK < 32 ? 32 : TOK;
-    static constexpr uint32_t A_COL0 = NACC * ACC_STRIDE;       // first TMEM column of the A ring
     static constexpr uint32_t X_BYTES = TOK * BK * 2;
     static constexpr uint32_t OFF_WB = 0;                       // S x 16 KB converted weights
-    static constexpr uint32_t OFF_X = OFF_WB + (A_TMEM ? 0u : S * WB_BYTES);   // S x tokens
+    static constexpr uint32_t OFF_X = OFF_WB + S * WB_BYTES;    // S x tokens
     static constexpr uint32_t OFF_WP = OFF_X + S * X_BYTES;     // PS x 4 KB packed weights
     static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES; // epilogue staging, 4 KB / warp
     static constexpr uint32_t OFF_BAR = OFF_EPI + 4096 * kEpiWarps;
-    static constexpr uint32_t BAR_BYTES = 8 * (2 * S + 2 * PS + 2 * NACC + 4) + 16;
-    static constexpr uint32_t OFF_SC = (OFF_BAR + BAR_BYTES + 127u) & ~127u;   // scale ring
-    // shared memory without the scale ring (+ slack for aligning the base to 1 KB)
-    static constexpr uint32_t SMEM_FIXED = OFF_SC + 1024;
+    static constexpr uint32_t BAR_BYTES = 8 * (2 * S + 2 * PS + 2 * NACC) + 16;
+    // + slack for aligning the base to 1 KB
+    static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
     static_assert(X_BYTES % 1024 == 0, "1 KB aligned stages");
     // a ring slot is only ever used by one converter group, so that the parity
     // waits and the per-group arrival counts never mix two groups' steps
     static_assert(S % kConvGroups == 0 && PS % kConvGroups == 0, "rings split over groups");
-    static_assert(NACC == 1 || NACC == 2, "one or two accumulators");
-    static_assert((A_TMEM ? A_COL0 + S * (BK / 2) : NACC * ACC_STRIDE) <= TMEM_COLS, "TMEM columns");
+    static_assert(NACC * ACC_STRIDE <= TMEM_COLS, "TMEM columns");
     static_assert(TOK % 32 == 0 && TOK <= 256, "token tile");
-    // bytes of one scale-ring slot for K/32 scale bytes per row (0 without A_TMEM)
-    __host__ __device__ static constexpr uint32_t sc_slot_bytes(int kblocks) {
-        return A_TMEM ? ((uint32_t)(BM * kblocks) + 127u) & ~127u : 0u;
-    }
-    __host__ __device__ static constexpr uint32_t smem_bytes(int kblocks) {
-        return SMEM_FIXED + 2 * sc_slot_bytes(kblocks);
-    }
+    __host__ __device__ static constexpr uint32_t smem_bytes(int /*kblocks*/) { return SMEM_BYTES; }
 };
-#ifndef MOE_PREFILL_TMEM_TOK
-#define MOE_PREFILL_TMEM_TOK 256
-#endif
-#ifndef MOE_PREFILL_TMEM_NACC
-#define MOE_PREFILL_TMEM_NACC 1
-#endif
-#ifndef MOE_PREFILL_TMEM_PS
-#define MOE_PREFILL_TMEM_PS 8
-#endif
-#ifndef MOE_DECODE_TMEM_S
-#define MOE_DECODE_TMEM_S 12
-#endif
-#ifndef MOE_DECODE_TMEM_PS
-#define MOE_DECODE_TMEM_PS 24
-#endif
 using PrefillCfg = Config<256, 4, 4>;
 using DecodeCfg = Config<32, 8, 8>;
-using PrefillTmemCfg = Config<MOE_PREFILL_TMEM_TOK, 4, MOE_PREFILL_TMEM_PS, true, MOE_PREFILL_TMEM_NACC>;
-using DecodeTmemCfg = Config<32, MOE_DECODE_TMEM_S, MOE_DECODE_TMEM_PS, true, 2>;
 
 struct Params {
     const int32_t *counts;        // [E]
@@ -213,8 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto x_stage = [&](int s) { return base + Cfg::OFF_X + s * Cfg::X_BYTES; };
     auto wp_stage = [&](int s) { return base + Cfg::OFF_WP + s * WP_BYTES; };
     const int kblocks = p.K / 32;
-    const uint32_t sc_slot = Cfg::sc_slot_bytes(kblocks);
-    auto sc_stage = [&](int b) { return base + Cfg::OFF_SC + b * sc_slot; };
     const uint32_t bars = base + Cfg::OFF_BAR;
     // ready(s): the token tile landed (producer arrival + transaction bytes) and
     // every converter warp of the step's group stored its weights
@@ -224,10 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wp_empty = [&](int s) { return bars + 8u * (2 * S + PS + s); };
     auto a_full = [&](int b) { return bars + 8u * (2 * S + 2 * PS + b); };
     auto a_empty = [&](int b) { return bars + 8u * (2 * S + 2 * PS + Cfg::NACC + b); };
-    // scale ring (A_TMEM): a tile's E8M0 bytes landed / every converter warp is done with them
-    auto sc_full = [&](int b) { return bars + 8u * (2 * S + 2 * PS + 2 * Cfg::NACC + b); };
-    auto sc_empty = [&](int b) { return bars + 8u * (2 * S + 2 * PS + 2 * Cfg::NACC + 2 + b); };
-    const uint32_t tmem_holder = bars + 8u * (2 * S + 2 * PS + 2 * Cfg::NACC + 4);
+    const uint32_t tmem_holder = bars + 8u * (2 * S + 2 * PS + 2 * Cfg::NACC);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -242,10 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < Cfg::NACC; ++b) {
             ptx::mbar_init(a_full(b), 1);
             ptx::mbar_init(a_empty(b), kEpiWarps);
-        }
-        for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(sc_full(b), 1);
-            ptx::mbar_init(sc_empty(b), kConvWarps);
         }
         ptx::fence_mbarrier_init();
         ptx::prefetch_tmap(&tmap_x);
@@ -290,21 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kWpWarp) {
         // ------------------------------------------------------------ packed-weight TMA
-        uint32_t it = 0, local = 0;
+        uint32_t it = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
             const Tile t = decode_tile<TOK>(p, item, w_tiles);
-            if constexpr (Cfg::A_TMEM) {
-                // the tile's scale rows, contiguous in [E, N, K/32]
-                const int b = local & 1;
-                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(sc_empty(b), ((local >> 1) & 1u) ^ 1u)))) break;
-                if (ptx::elect_one()) {
-                    const uint32_t bytes = (uint32_t)(t.mrows * kblocks);
-                    ptx::mbar_arrive_expect_tx(sc_full(b), bytes);
-                    ptx::bulk_load(sc_stage(b), p.wscales + ((int64_t)t.e * p.N + t.m0) * kblocks, bytes, sc_full(b));
-                }
-                __syncwarp();
-            }
             for (int kb = 0; kb < k_iters; ++kb, ++it) {
                 const int s = it % PS;
                 if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_empty(s), ((it / PS) & 1u) ^ 1u)))) break;
@@ -335,18 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_after();
                 const uint64_t bd = ptx::sw128_kmajor_desc(x_stage(s));
                 if (ptx::elect_one()) {
-                    if constexpr (Cfg::A_TMEM) {
-                        const uint32_t a_tmem = tmem_base + Cfg::A_COL0 + s * (BK / 2);
+                    const uint64_t ad = ptx::sw128_kmajor_desc(wb_stage(s));
 #pragma unroll
-                        for (int j = 0; j < BK / 16; ++j)   // 8 TMEM columns / +32 B per 16-element K step
-                            ptx::mma_bf16_ta(d_tmem, a_tmem + 8u * j, bd + 2u * j, idesc,
-                                             (kb > 0 || j > 0) ? 1u : 0u);
-                    } else {
-                        const uint64_t ad = ptx::sw128_kmajor_desc(wb_stage(s));
-#pragma unroll
-                        for (int j = 0; j < BK / 16; ++j)   // +32 B per 16-element K step (start address >> 4)
-                            ptx::mma_bf16(d_tmem, ad + 2u * j, bd + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
-                    }
+                    for (int j = 0; j < BK / 16; ++j)   // +32 B per 16-element K step (start address >> 4)
+                        ptx::mma_bf16(d_tmem, ad + 2u * j, bd + 2u * j, idesc, (kb > 0 || j > 0) ? 1u : 0u);
                     ptx::mma_commit(empty(s));
                 }
                 __syncwarp();
@@ -443,78 +379,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(a_empty(b));
-        }
-    } else if constexpr (Cfg::A_TMEM) {
-        // ------------------------------------------------------------ converters (A in TMEM)
-        // Warp w may only touch TMEM lanes 32 (w % 4) .. +31, so each converter thread
-        // owns one weight row (lane) and turns that row's 64 codes of a step (two
-        // 32-element blocks, 32 bytes) into 32 bf16x2 columns; a group's four
-        // consecutive warps cover the four lane quarters.  Conversion as in the
-        // shared-memory variant below; the E8M0 bytes come from the tile's scale slot.
-        const int grp = (warp - kFirstConvWarp) / (kConvWarps / kConvGroups);
-        const int q = warp & 3;
-        const int row = q * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        uint32_t it = 0, local = 0;
-        bool ok = true;
-        for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
-            const int sb = local & 1;
-            // every converter warp takes part in every tile's scale slot, even with no
-            // step of its own in the tile, so the slot's arrival count never mixes tiles
-            if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(sc_full(sb), (local >> 1) & 1u)))) break;
-            // out-of-range rows read the slot's unused tail; their codes are zero-filled
-            const uint32_t sc_row = sc_stage(sb) + (uint32_t)(row < t.mrows ? row : 0) * (uint32_t)kblocks;
-            for (int kb = (int)((grp - (int)(it % kConvGroups) + kConvGroups) % kConvGroups); kb < k_iters;
-                 kb += kConvGroups) {
-                const uint32_t gi = it + (uint32_t)kb;         // global step index
-                const int c = gi % S, ps = gi % PS;
-                const uint32_t sc2 = ptx::ld_shared_u16(sc_row + 2 * kb);
-                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (gi / PS) & 1u)))) break;
-                const uint4 qa = ptx::ld_shared_v4(wp_stage(ps) + row * 32);
-                const uint4 qb = ptx::ld_shared_v4(wp_stage(ps) + row * 32 + 16);
-                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(c), ((gi / S) & 1u) ^ 1u)))) break;
-                ptx::tc_fence_after();
-                uint32_t v[32];
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const uint32_t sc = blk ? (sc2 >> 8) : (sc2 & 0xFFu);
-                    uint32_t m1, m2 = 0;
-                    if (sc == 255u) {
-                        raise_device_error(MOE_DEVERR_BAD_SCALE);
-                        m1 = 0x7FC07FC0u;
-                    } else if (sc <= 128u) {
-                        m1 = ((sc + 126u) << 7) * 0x10001u;
-                    } else {
-                        m1 = 0x7E807E80u;
-                        m2 = (sc << 7) * 0x10001u;
-                    }
-                    const uint4 qv = blk ? qb : qa;
-                    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        uint32_t r[4];
-                        e2m1x8_to_bf16_rep(qw[w], r[0], r[1], r[2], r[3]);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            r[j] = ptx::hmul2_bf16(r[j], m1);
-                            if (m2) r[j] = ptx::hmul2_bf16(r[j], m2);
-                            v[blk * 16 + w * 4 + j] = r[j];
-                        }
-                    }
-                }
-                ptx::tmem_st_32x32b_x32(tmem_base + lane_off + Cfg::A_COL0 + c * (BK / 2), v);
-                ptx::tmem_st_wait();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(ready(c));
-                    ptx::mbar_arrive(wp_empty(ps));
-                }
-            }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(sc_empty(sb));
-            it += (uint32_t)k_iters;
         }
     } else {
         // ------------------------------------------------------------ converters

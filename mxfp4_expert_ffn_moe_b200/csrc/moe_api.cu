@@ -353,17 +353,10 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
 // average, 256-row tiles otherwise.
 bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
 
-#ifndef MOE_DECODE_A_TMEM
-#define MOE_DECODE_A_TMEM 1
-#endif
-#ifndef MOE_PREFILL_A_TMEM
-#define MOE_PREFILL_A_TMEM 0
-#endif
-
-// Tile configurations of the grouped GEMMs.  The TMEM-operand variants hold two
-// tiles' scale rows (128 x K/32 bytes each) in shared memory; for K too large for
-// that they give way to the shared-memory-operand variant of the same tiles.
-enum TileConfig { kDecodeSmem, kDecodeTmem, kPrefillSmem, kPrefillTmem, kDecodeMxf, kPrefillMxf };
+// Tile configurations of the grouped GEMMs: the block-scaled kernel (decode tiles) holds
+// two tiles' scale rows (128 x K/32 bytes each) in shared memory; for K too large for
+// that, the converter kernel's 32-token tiles take over.
+enum TileConfig { kDecodeSmem, kPrefillSmem, kDecodeMxf, kPrefillMxf };
 
 #ifndef MOE_MXF_DECODE
 #define MOE_MXF_DECODE 1
@@ -379,21 +372,17 @@ bool config_fits(int64_t H, int64_t I) {
 }
 
 TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E) {
-    if (use_decode_tiles(P, E) && MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) return kDecodeMxf;
-    if (!use_decode_tiles(P, E) && MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) return kPrefillMxf;
     if (use_decode_tiles(P, E))
-        return (MOE_DECODE_A_TMEM && config_fits<moe::swp::DecodeTmemCfg>(H, I)) ? kDecodeTmem : kDecodeSmem;
-    return (MOE_PREFILL_A_TMEM && config_fits<moe::swp::PrefillTmemCfg>(H, I)) ? kPrefillTmem : kPrefillSmem;
+        return (MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) ? kDecodeMxf : kDecodeSmem;
+    return (MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) ? kPrefillMxf : kPrefillSmem;
 }
 
 int config_tok(TileConfig c) {
     switch (c) {
         case kDecodeSmem: return moe::swp::DecodeCfg::TOK;
-        case kDecodeTmem: return moe::swp::DecodeTmemCfg::TOK;
         case kPrefillSmem: return moe::swp::PrefillCfg::TOK;
         case kDecodeMxf: return moe::mxf::DecodeCfg::TOK;
-        case kPrefillMxf: return moe::mxf::PrefillCfg::TOK;
-        default: return moe::swp::PrefillTmemCfg::TOK;
+        default: return moe::mxf::PrefillCfg::TOK;
     }
 }
 
@@ -539,12 +528,7 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
     launch_projections<C>(x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias, \
                           down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,         \
                           tile_offsets, sorted_pairs, weights, woi, s)
-            switch (cfg) {
-                case kDecodeSmem: rc = MOE_PROJECTIONS(moe::swp::DecodeCfg); break;
-                case kDecodeTmem: rc = MOE_PROJECTIONS(moe::swp::DecodeTmemCfg); break;
-                case kPrefillSmem: rc = MOE_PROJECTIONS(moe::swp::PrefillCfg); break;
-                default: rc = MOE_PROJECTIONS(moe::swp::PrefillTmemCfg); break;
-            }
+            rc = cfg == kDecodeSmem ? MOE_PROJECTIONS(moe::swp::DecodeCfg) : MOE_PROJECTIONS(moe::swp::PrefillCfg);
 #undef MOE_PROJECTIONS
         }
         if (rc != MOE_OK) break;

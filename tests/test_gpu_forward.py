@@ -70,6 +70,8 @@ def test_tiny_layers_full_compare(moe_gpu, oracle_mod, name):
     (130, 128, 64, 3, 2, True),      # more than two M tiles per expert, weight on input
     (3, 256, 128, 16, 4, False),     # most experts empty
     (200, 64, 128, 2, 2, False),     # every pair on the same two experts
+    (3, 8192, 64, 4, 2, False),      # decode tiles with K = 8192: the block-scaled kernel's two
+                                     # tile scale slots do not fit, the converter kernel serves
 ])
 def test_edge_shapes(moe_gpu, oracle_mod, T, H, I, E, k, woi):
     layer = make_layer(T, H, I, E, k, seed=T + H, biases=not woi, weight_on_input=woi,
