@@ -13,6 +13,11 @@ Recipe (every array from ``numpy.random.default_rng(seed)``, drawn in this order
               codes per byte), E8M0 scales uint8 [E, 2I, H/32] uniform in
               [scale_lo, scale_hi], bias fp32 [E, 2I] N(0, bias_std^2), bias_std = 0.02
 * down        packed uint8 [E, H, I/2], scales [E, H, I/32], bias fp32 [E, H], same laws
+
+NVFP4 layers (``fmt="nvfp4"``) draw in the same order with one E4M3 scale byte per 16
+elements ([E, N, K/16], uniform in [e4m3_lo, e4m3_hi] = [0x08, 0x37]: 2^-6 .. 0.9375,
+sign clear), then append the per-expert fp32 weight_scale_2 draws: gate_up [E, 2]
+(gate, up) and down [E], uniform in [0.5, 1).
 """
 from __future__ import annotations
 
@@ -35,9 +40,11 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 @dataclass
 class ExpertBank:
-    """One packed MXFP4 projection bank: blocks [E, N, K/2], scales [E, N, K/32]."""
+    """One packed projection bank: blocks [E, N, K/2] and scales, E8M0 [E, N, K/32]
+    (MXFP4) or E4M3 [E, N, K/16] with a per-expert fp32 ``scale2`` (NVFP4)."""
     blocks: np.ndarray
     scales: np.ndarray
+    scale2: Optional[np.ndarray] = None
 
     @property
     def shape(self):
@@ -62,19 +69,26 @@ class MoELayer:
     limit: float = 7.0
     weight_on_input: bool = False
     name: str = field(default="")
+    fmt: str = "mxfp4"
+
+
+E4M3_LO, E4M3_HI = 0x08, 0x37
 
 
 def make_bank(rng: np.random.Generator, E: int, N: int, K: int, scale_lo: int,
-              scale_hi: int) -> ExpertBank:
+              scale_hi: int, block: int = 32) -> ExpertBank:
     blocks = rng.integers(0, 256, size=(E, N, K // 2), dtype=np.uint8)
-    scales = rng.integers(scale_lo, scale_hi + 1, size=(E, N, K // 32), dtype=np.uint8)
+    scales = rng.integers(scale_lo, scale_hi + 1, size=(E, N, K // block), dtype=np.uint8)
     return ExpertBank(blocks, scales)
 
 
 def make_layer(T: int, H: int, I: int, E: int, k: int, seed: int = 0, scale_lo: int = 118,
                scale_hi: int = 126, zipf: float = 0.0, biases: bool = True,
                weight_on_input: bool = False, bias_std: float = 0.02,
-               name: str = "") -> MoELayer:
+               name: str = "", fmt: str = "mxfp4") -> MoELayer:
+    assert fmt in ("mxfp4", "nvfp4")
+    if fmt == "nvfp4":
+        return _make_nvfp4_layer(T, H, I, E, k, seed, zipf, biases, weight_on_input, bias_std, name)
     rng = np.random.default_rng(seed)
     x_bits = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
     logits = rng.standard_normal((T, E), dtype=np.float32)
@@ -90,6 +104,36 @@ def make_layer(T: int, H: int, I: int, E: int, k: int, seed: int = 0, scale_lo: 
         d_bias = None
     return MoELayer(T, H, I, E, k, x_bits, logits, gu, gu_bias, dn, d_bias,
                     weight_on_input=weight_on_input, name=name)
+
+
+def _make_nvfp4_layer(T, H, I, E, k, seed, zipf, biases, weight_on_input, bias_std, name):
+    rng = np.random.default_rng(seed)
+    x_bits = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    logits = rng.standard_normal((T, E), dtype=np.float32)
+    if zipf:
+        rank = np.arange(1, E + 1, dtype=np.float64)
+        logits = (logits + (zipf * np.log(1.0 / rank)).astype(np.float32)[None, :]).astype(np.float32)
+    gu = make_bank(rng, E, 2 * I, H, E4M3_LO, E4M3_HI, block=16)
+    gu_bias = (bias_std * rng.standard_normal((E, 2 * I))).astype(np.float32)
+    dn = make_bank(rng, E, H, I, E4M3_LO, E4M3_HI, block=16)
+    d_bias = (bias_std * rng.standard_normal((E, H))).astype(np.float32)
+    gu.scale2 = rng.uniform(0.5, 1.0, size=(E, 2)).astype(np.float32)
+    dn.scale2 = rng.uniform(0.5, 1.0, size=(E,)).astype(np.float32)
+    if not biases:
+        gu_bias = None
+        d_bias = None
+    return MoELayer(T, H, I, E, k, x_bits, logits, gu, gu_bias, dn, d_bias,
+                    weight_on_input=weight_on_input, name=name, fmt="nvfp4")
+
+
+def make_nvfp4_dequant_bank(seed: int = 0, E: int = 32, H: int = 2880, I: int = 2880):
+    """gpt-oss-20b-shaped NVFP4 expert bank for the standalone dequant workload."""
+    rng = np.random.default_rng(seed)
+    gu = make_bank(rng, E, 2 * I, H, E4M3_LO, E4M3_HI, block=16)
+    dn = make_bank(rng, E, H, I, E4M3_LO, E4M3_HI, block=16)
+    gu.scale2 = rng.uniform(0.5, 1.0, size=(E,)).astype(np.float32)
+    dn.scale2 = rng.uniform(0.5, 1.0, size=(E,)).astype(np.float32)
+    return gu, dn
 
 
 def make_dequant_bank(seed: int = 0, E: int = 32, H: int = 2880, I: int = 2880,
@@ -114,6 +158,14 @@ WORKLOADS = {
     "20b_prefill_T4096": dict(T=4096, H=2880, I=2880, E=32, k=4),
     "120b_zipf_T256": dict(T=256, H=2880, I=2880, E=128, k=4, zipf=1.5),
     "120b_zipf_T8192": dict(T=8192, H=2880, I=2880, E=128, k=4, zipf=1.5),
+    # the NVFP4 expert variant of the same layers
+    "nvfp4_tiny_woo": dict(T=8, H=128, I=128, E=4, k=2, biases=True, fmt="nvfp4"),
+    "nvfp4_tiny_woi": dict(T=8, H=128, I=128, E=4, k=2, biases=False, weight_on_input=True,
+                           fmt="nvfp4"),
+    "nvfp4_tiny_bias_heavy": dict(T=8, H=128, I=128, E=4, k=2, biases=True, bias_std=8.0,
+                                  fmt="nvfp4"),
+    "nvfp4_20b_decode_T8": dict(T=8, H=2880, I=2880, E=32, k=4, fmt="nvfp4"),
+    "nvfp4_20b_prefill_T4096": dict(T=4096, H=2880, I=2880, E=32, k=4, fmt="nvfp4"),
 }
 
 

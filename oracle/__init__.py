@@ -16,6 +16,10 @@ What each entry point follows is cited in ``moe_oracle.c``; in short:
 * ``forward_tokens`` / ``forward_grouped`` -- FreeToken PR #838 "feat(gguf): serve
   gpt-oss gguf checkpoints on gpt_oss", review items on the down bias and on
   apply_router_weight_on_input, and "What it does" (alpha 1.702, limit 7, bias roles).
+* ``e4m3_value`` / ``nvfp4_dequantize`` / ``nvfp4_forward_tokens`` -- the NVFP4 expert
+  variant: E2M1 codes with one E4M3 scale per 16 elements (OCP OFP8 v1.0 for E4M3)
+  and a per-expert fp32 weight_scale_2 that multiplies each projection before its
+  bias (FreeToken PR #838, review item "NVFP4 down scale vs. down bias").
 
 Every function here is pinned by the CPU tests against hand-written values, closed
 forms, invariants or a library routine; none is "parity unpinned".
@@ -41,6 +45,9 @@ DEFECT_UNINTERLEAVED = 5
 DEFECT_DOWN_BIAS_UNWEIGHTED = 6
 DEFECT_WOI_BIAS_WEIGHTED = 7
 DEFECT_DOWN_BIAS_IN_SCALE = 8
+DEFECT_NVFP4_SCALE_AFTER_BIAS = 9
+DEFECT_NVFP4_BLOCK32 = 10
+DEFECT_NVFP4_GU_SCALE_SWAP = 11
 
 FLAG_WEIGHT_ON_INPUT = 1
 
@@ -86,6 +93,15 @@ def _load():
         lib.oracle_forward_grouped.argtypes = [p, i64, i64, i64, i64, ctypes.c_int, p, p,
                                                p, p, p, p, p, p, ctypes.c_double, ctypes.c_double,
                                                ctypes.c_int, p]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_int]
+        lib.oracle_nvfp4_dequantize.restype = None
+        lib.oracle_nvfp4_dequantize.argtypes = [p, p, p, p, i64, i64, i64, ctypes.c_int]
+        lib.oracle_nvfp4_forward_tokens.restype = None
+        lib.oracle_nvfp4_forward_tokens.argtypes = [p, i64, i64, i64, i64, ctypes.c_int, p, p,
+                                                    p, p, p, p, p, p, p, p, ctypes.c_double,
+                                                    ctypes.c_double, ctypes.c_int, p, i64, p, p,
+                                                    ctypes.c_int]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -187,6 +203,57 @@ def forward_grouped(x_bits, ids, weights, gu_blocks, gu_scales, gu_bias, d_block
     if rc != 0:
         raise MemoryError("oracle_forward_grouped: allocation failed")
     return out
+
+
+def e4m3_value(b: int) -> float:
+    return _load().oracle_e4m3_value(int(b))
+
+
+def nvfp4_dequantize(blocks, scales, scale2, E: int, N: int, K: int,
+                     defect: int = DEFECT_NONE) -> np.ndarray:
+    """Packed [E,N,K/2] + E4M3 [E,N,K/16] (+ fp32 [E] or None) -> bf16 bits uint16 [E,N,K]."""
+    blocks = _c(blocks, np.uint8)
+    scales = _c(scales, np.uint8)
+    scale2 = _c(scale2, np.float32)
+    assert blocks.size == E * N * K // 2 and scales.size == E * N * K // 16
+    assert scale2 is None or scale2.size == E
+    out = np.empty((E, N, K), dtype=np.uint16)
+    _load().oracle_nvfp4_dequantize(_ptr(blocks), _ptr(scales), _ptr(scale2), _ptr(out), E, N, K,
+                                    int(defect))
+    return out
+
+
+def nvfp4_forward_tokens(x_bits, ids, weights, gu_blocks, gu_scales, gu_scale2, gu_bias,
+                         d_blocks, d_scales, d_scale2, d_bias, alpha=1.702, limit=7.0,
+                         weight_on_input=False, tokens=None, defect: int = DEFECT_NONE,
+                         envelope: bool = False):
+    """Formulation A with NVFP4 experts.  gu_scale2 fp32 [E, 2] (gate, up) and d_scale2
+    fp32 [E] may be None (1).  Returns float64 [len(tokens), H] (and the envelope)."""
+    x_bits = _c(x_bits, np.uint16)
+    T, H = x_bits.shape
+    ids = _c(ids, np.int32)
+    k = ids.shape[1]
+    weights = _c(weights, np.float32)
+    gu_blocks = _c(gu_blocks, np.uint8)
+    E = gu_blocks.shape[0]
+    I = gu_blocks.shape[1] // 2
+    gu_scale2 = _c(gu_scale2, np.float32)
+    d_scale2 = _c(d_scale2, np.float32)
+    assert gu_scale2 is None or gu_scale2.size == 2 * E
+    assert d_scale2 is None or d_scale2.size == E
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int64)
+    tokens = _c(tokens, np.int64)
+    out = np.empty((tokens.size, H), dtype=np.float64)
+    env = np.empty((tokens.size, H), dtype=np.float64) if envelope else None
+    _load().oracle_nvfp4_forward_tokens(
+        _ptr(x_bits), T, H, I, E, k, _ptr(ids), _ptr(weights), _ptr(gu_blocks),
+        _ptr(_c(gu_scales, np.uint8)), _ptr(gu_scale2), _ptr(_c(gu_bias, np.float32)),
+        _ptr(_c(d_blocks, np.uint8)), _ptr(_c(d_scales, np.uint8)), _ptr(d_scale2),
+        _ptr(_c(d_bias, np.float32)), float(alpha), float(limit),
+        FLAG_WEIGHT_ON_INPUT if weight_on_input else 0, _ptr(tokens), tokens.size, _ptr(out),
+        _ptr(env), int(defect))
+    return (out, env) if envelope else out
 
 
 def num_threads() -> int:

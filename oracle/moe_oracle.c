@@ -29,6 +29,12 @@
  *   [MX] OCP Microscaling Formats (MX) v1.0: FP4 E2M1 element (1 sign, 2 exponent
  *        bits with bias 1, 1 mantissa bit, no inf/NaN) and E8M0 scale (2^(b-127),
  *        0xff = NaN).
+ *   [F8] OCP 8-bit Floating Point Specification (OFP8) v1.0: the E4M3 format (1 sign,
+ *        4 exponent bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 NaN,
+ *        largest magnitude 448).
+ *   [N4] NVFP4 as NVIDIA publishes it: blocks of 16 E2M1 elements sharing one E4M3
+ *        scale, plus one fp32 scale per tensor ("weight_scale_2"); [P3] review item
+ *        "NVFP4 down scale vs. down bias" fixes where that fp32 scale enters.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   R1  element kk of a packed row lives in byte kk/2; the LOW nibble holds the
@@ -40,6 +46,13 @@
  *   R4  clamped SwiGLU: g = min(gate, limit), u = clamp(up, -limit, limit),
  *       a = (u + 1) * g * sigmoid(alpha * g).
  *   R5  a 0xff scale byte decodes to NaN (the pages reject it as invalid).
+ *   R6  NVFP4 experts: W[e, n, kk] = E2M1(code) * E4M3(scale[e, n, kk/16]) with the
+ *       packing of R1; each projection's fp32 weight_scale_2 multiplies the expert's
+ *       matrix product before its bias is added (h = s*acc + b, y = s*acc + b).  The
+ *       fused gate_up bank carries two per expert (gate rows, up rows: index 0 and 1
+ *       of the per-expert triple the review indexes, down being index 2).
+ *   R7  the standalone NVFP4 dequant returns bf16 rounded once (nearest, ties to even)
+ *       from the exact product E2M1 * E4M3 * weight_scale_2.
  *
  * Function that is not pinned by anything outside itself: none -- every entry
  * point is checked against hand-written values, closed forms, invariants or a
@@ -63,7 +76,15 @@ enum {
                                                by the routing weight                  */
     ORACLE_DEFECT_DOWN_BIAS_IN_SCALE = 8,   /* down bias multiplied by the row's first
                                                E8M0 block scale (scale after bias)    */
+    ORACLE_DEFECT_NVFP4_SCALE_AFTER_BIAS = 9, /* NVFP4: y = s*(acc + b), the mistake the
+                                                 [P3] review item describes           */
+    ORACLE_DEFECT_NVFP4_BLOCK32 = 10,       /* NVFP4: one scale per 32 elements (the
+                                               first 16-block's scale for both halves) */
+    ORACLE_DEFECT_NVFP4_GU_SCALE_SWAP = 11, /* NVFP4: gate rows take the up scale and
+                                               the other way round                    */
 };
+
+enum { ORACLE_FMT_MXFP4 = 0, ORACLE_FMT_NVFP4 = 1 };
 
 enum { ORACLE_FLAG_WEIGHT_ON_INPUT = 1 };
 
@@ -90,6 +111,24 @@ double oracle_e8m0_value(int b, int defect)
     if (b == 255)
         return NAN;
     return ldexp(1.0, b - (defect == ORACLE_DEFECT_E8M0_BIAS_126 ? 126 : 127));
+}
+
+/* E4M3 [F8]: bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0 mantissa.
+ * Exponent field 0 is subnormal: magnitude = m/8 * 2^-6.  Exponent and mantissa
+ * all ones is NaN (there are no infinities). */
+double oracle_e4m3_value(int b)
+{
+    int sign = (b >> 7) & 1;
+    int e = (b >> 3) & 15;
+    int m = b & 7;
+    double mag;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, -6);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
 }
 
 /* double -> bfloat16 bits, round to nearest, ties to even, with subnormals
@@ -144,6 +183,49 @@ static double weight_elem(const uint8_t *blocks, const uint8_t *scales,
     int code = even ? (byte & 0xF) : (byte >> 4);
     int s = scales[row * (K / 32) + kk / 32];
     return oracle_e2m1_value(code) * oracle_e8m0_value(s, defect);
+}
+
+/* One weight element of a packed NVFP4 bank (reading R6): blocks [E, N, K/2] with
+ * the nibble order of R1, E4M3 scales [E, N, K/16], one per 16 elements [N4]. */
+static double weight_elem_nvfp4(const uint8_t *blocks, const uint8_t *scales,
+                                int64_t N, int64_t K, int64_t e, int64_t n, int64_t kk,
+                                int defect)
+{
+    int64_t row = e * N + n;
+    uint8_t byte = blocks[row * (K / 2) + kk / 2];
+    int even = (kk % 2) == 0;
+    if (defect == ORACLE_DEFECT_NIBBLE_SWAP)
+        even = !even;
+    int code = even ? (byte & 0xF) : (byte >> 4);
+    int64_t blk = kk / 16;
+    if (defect == ORACLE_DEFECT_NVFP4_BLOCK32)
+        blk = (kk / 32) * 2;
+    return oracle_e2m1_value(code) * oracle_e4m3_value(scales[row * (K / 16) + blk]);
+}
+
+static double weight_elem_fmt(int fmt, const uint8_t *blocks, const uint8_t *scales,
+                              int64_t N, int64_t K, int64_t e, int64_t n, int64_t kk,
+                              int defect)
+{
+    if (fmt == ORACLE_FMT_NVFP4)
+        return weight_elem_nvfp4(blocks, scales, N, K, e, n, kk, defect);
+    return weight_elem(blocks, scales, N, K, e, n, kk, defect);
+}
+
+/* NVFP4 dequant (reading R7): out[e, n, kk] = bf16(E2M1 * E4M3 * s2[e]), s2 = 1
+ * when scale2 is NULL.  E2M1 * E4M3 has at most 6 significant bits, so the product
+ * with an fp32 s2 (24 bits) is exact in double and oracle_double_to_bf16 rounds it
+ * once. */
+void oracle_nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2,
+                             uint16_t *out, int64_t E, int64_t N, int64_t K, int defect)
+{
+    for (int64_t e = 0; e < E; ++e) {
+        double s2 = scale2 ? (double)scale2[e] : 1.0;
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t kk = 0; kk < K; ++kk)
+                out[(e * N + n) * K + kk] = oracle_double_to_bf16(
+                    weight_elem_nvfp4(blocks, scales, N, K, e, n, kk, defect) * s2);
+    }
 }
 
 /* ---- standalone dequant-on-copy [P2] Changes ------------------------------- */
@@ -225,14 +307,17 @@ double oracle_swiglu(double gate, double up, double alpha, double limit, int def
  *   the input).  It bounds |out| by the triangle inequality and scales the error a
  *   rounded activation operand can cause (MoE-Infinity PR #152, Changes: the parity
  *   test pairs an fp32 golden with a magnitude envelope). */
-void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
-                           int64_t E, int k, const int32_t *ids, const float *w,
-                           const uint8_t *gu_blocks, const uint8_t *gu_scales,
-                           const float *gu_bias, const uint8_t *d_blocks,
-                           const uint8_t *d_scales, const float *d_bias,
-                           double alpha, double limit, int flags,
-                           const int64_t *token_list, int64_t n_list, double *out,
-                           double *env, int defect)
+/* fmt selects the weight format; gu_s2 [E, 2] (gate, up) and d_s2 [E] are the
+ * NVFP4 per-expert fp32 scales (NULL: 1), unused for MXFP4. */
+static void forward_tokens_impl(int fmt, const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                                int64_t E, int k, const int32_t *ids, const float *w,
+                                const uint8_t *gu_blocks, const uint8_t *gu_scales,
+                                const float *gu_s2, const float *gu_bias,
+                                const uint8_t *d_blocks, const uint8_t *d_scales,
+                                const float *d_s2, const float *d_bias,
+                                double alpha, double limit, int flags,
+                                const int64_t *token_list, int64_t n_list, double *out,
+                                double *env, int defect)
 {
     (void)T;
     (void)E;
@@ -264,8 +349,16 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
                     zero_row = (n % 2) == 0; /* interleaved: even rows are gate */
                 if (!zero_row)
                     for (int64_t c = 0; c < H; ++c)
-                        acc += xin[c] * weight_elem(gu_blocks, gu_scales, N_gu, H, e, n, c, defect);
-                h[n] = acc + (gu_bias ? (double)gu_bias[e * N_gu + n] : 0.0);
+                        acc += xin[c] * weight_elem_fmt(fmt, gu_blocks, gu_scales, N_gu, H, e, n, c, defect);
+                /* NVFP4: the row's weight_scale_2 before the bias (reading R6) */
+                double s2 = 1.0;
+                if (fmt == ORACLE_FMT_NVFP4 && gu_s2) {
+                    int role = (int)(n % 2); /* 0 gate, 1 up (reading R3) */
+                    if (defect == ORACLE_DEFECT_NVFP4_GU_SCALE_SWAP)
+                        role = 1 - role;
+                    s2 = (double)gu_s2[e * 2 + role];
+                }
+                h[n] = s2 * acc + (gu_bias ? (double)gu_bias[e * N_gu + n] : 0.0);
             }
             for (int64_t i = 0; i < I; ++i) {
                 double gate, up;
@@ -282,11 +375,17 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
             for (int64_t c = 0; c < H; ++c) {
                 double acc = 0.0, mag = 0.0;
                 for (int64_t i = 0; i < I; ++i) {
-                    double term = a[i] * weight_elem(d_blocks, d_scales, H, I, e, c, i, defect);
+                    double term = a[i] * weight_elem_fmt(fmt, d_blocks, d_scales, H, I, e, c, i, defect);
                     acc += term;
                     mag += fabs(term);
                 }
                 double b = d_bias ? (double)d_bias[e * H + c] : 0.0;
+                /* NVFP4: y = s*acc + b (reading R6; [P3] NVFP4 down scale vs. down bias) */
+                double s2 = (fmt == ORACLE_FMT_NVFP4 && d_s2) ? (double)d_s2[e] : 1.0;
+                if (defect == ORACLE_DEFECT_NVFP4_SCALE_AFTER_BIAS)
+                    b *= s2;
+                acc *= s2;
+                mag *= fabs(s2);
                 if (ev)
                     ev[c] += (woi ? 1.0 : fabs(wj)) * (mag + fabs(b));
                 if (defect == ORACLE_DEFECT_DOWN_BIAS_IN_SCALE)
@@ -307,6 +406,38 @@ void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
         free(h);
         free(xin);
     }
+}
+
+void oracle_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                           int64_t E, int k, const int32_t *ids, const float *w,
+                           const uint8_t *gu_blocks, const uint8_t *gu_scales,
+                           const float *gu_bias, const uint8_t *d_blocks,
+                           const uint8_t *d_scales, const float *d_bias,
+                           double alpha, double limit, int flags,
+                           const int64_t *token_list, int64_t n_list, double *out,
+                           double *env, int defect)
+{
+    forward_tokens_impl(ORACLE_FMT_MXFP4, x, T, H, I, E, k, ids, w, gu_blocks, gu_scales, NULL,
+                        gu_bias, d_blocks, d_scales, NULL, d_bias, alpha, limit, flags,
+                        token_list, n_list, out, env, defect);
+}
+
+/* Formulation A for NVFP4 experts (reading R6): gu_scales E4M3 [E, 2I, H/16],
+ * gu_s2 fp32 [E, 2] (gate, up; NULL = 1), d_scales E4M3 [E, H, I/16], d_s2 fp32 [E]
+ * (NULL = 1).  Everything else as oracle_forward_tokens. */
+void oracle_nvfp4_forward_tokens(const uint16_t *x, int64_t T, int64_t H, int64_t I,
+                                 int64_t E, int k, const int32_t *ids, const float *w,
+                                 const uint8_t *gu_blocks, const uint8_t *gu_scales,
+                                 const float *gu_s2, const float *gu_bias,
+                                 const uint8_t *d_blocks, const uint8_t *d_scales,
+                                 const float *d_s2, const float *d_bias,
+                                 double alpha, double limit, int flags,
+                                 const int64_t *token_list, int64_t n_list, double *out,
+                                 double *env, int defect)
+{
+    forward_tokens_impl(ORACLE_FMT_NVFP4, x, T, H, I, E, k, ids, w, gu_blocks, gu_scales, gu_s2,
+                        gu_bias, d_blocks, d_scales, d_s2, d_bias, alpha, limit, flags,
+                        token_list, n_list, out, env, defect);
 }
 
 /* ---- formulation B: group pairs by expert over a pre-decoded bank ----------- */
