@@ -9,7 +9,9 @@
  *            with g = min(gate, limit);  y = a . W_d[e]^T + b_d[e];
  *   combine: out[t] = sum_j w[t,j] * y_j   (the bias sits inside the weight).
  * Expert weights are MXFP4: E2M1 codes packed two per byte (even element in the
- * low nibble) with one E8M0 scale byte per 32 consecutive elements of a row.
+ * low nibble) with one E8M0 scale byte per 32 consecutive elements of a row; the
+ * NVFP4 variant (E4M3 scale per 16 elements plus an fp32 weight_scale_2 per
+ * expert) has its own entry points, nvfp4_dequantize and moe_nvfp4_forward_ex.
  *
  * Sources, cited by page title and section:
  *   MoE-Infinity PR #152 "expert offloading Phase 2 -- MXFP4 dequant-on-copy
@@ -64,7 +66,8 @@ typedef enum {
 
 /* Device error bits reported by moe_get_device_error (ORed). */
 #define MOE_DEVERR_BAD_EXPERT_ID 0x1 /* an id outside [0, E) reached the layer      */
-#define MOE_DEVERR_BAD_SCALE 0x2     /* an E8M0 byte 0xff was decoded                */
+#define MOE_DEVERR_BAD_SCALE 0x2     /* an E8M0 byte 0xff, or an E4M3 NaN byte
+                                        (0x7f / 0xff), was decoded                  */
 #define MOE_DEVERR_TIMEOUT 0x4       /* a bounded pipeline wait gave up              */
 
 /* moe_mxfp4_forward_ex flags */
@@ -142,8 +145,54 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                          float limit, uint16_t *out, uint32_t flags, void *workspace,
                          size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace moe_mxfp4_forward_ex needs for these sizes (0 on bad sizes). */
+/* Bytes of workspace moe_mxfp4_forward_ex (and moe_nvfp4_forward_ex) needs for
+ * these sizes (0 on bad sizes). */
 size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int k);
+
+/*
+ * NVFP4 expert banks: the packed E2M1 codes of the MXFP4 layout with one E4M3 scale
+ * byte per 16 consecutive elements of a row (OCP OFP8 v1.0 E4M3: bias 7, 3 mantissa
+ * bits, subnormals m/8 * 2^-6, 0x7f / 0xff NaN, no infinities) and one fp32
+ * weight_scale_2 per expert and projection.  FreeToken PR #838, review item "NVFP4
+ * down scale vs. down bias": the fp32 scale multiplies the expert's matrix product
+ * before its bias, out = sum_j w_j * (s * y_j + b).
+ */
+
+/*
+ * nvfp4_dequantize -- standalone dequant of a packed NVFP4 bank to bf16.
+ *   blocks  uint8 [E, N, K/2]   E2M1 codes, element 2m in the low nibble of byte m
+ *   scales  uint8 [E, N, K/16]  E4M3 byte per 16 consecutive elements of a row
+ *   scale2  fp32  [E] or NULL   weight_scale_2 per expert (NULL = 1)
+ *   out     bf16  [E, N, K]     E2M1(code) * E4M3(scale) * scale2, rounded once to
+ *                               nearest even from the exact product (exact when
+ *                               scale2 is NULL or a power of two in range); NaN as
+ *                               0x7fc0; a NaN scale byte sets MOE_DEVERR_BAD_SCALE
+ * Sizes: E, N >= 1; K >= 16 and K % 16 == 0.  blocks and out must be 16-byte
+ * aligned, scale2 4-byte aligned.  Errors: MOE_ERR_INVALID_ARG for null pointers,
+ * sizes or alignment.
+ */
+int nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2,
+                     uint16_t *out, int64_t E, int64_t N, int64_t K, void *stream);
+
+/*
+ * moe_nvfp4_forward_ex -- the expert layer of moe_mxfp4_forward_ex over NVFP4 banks:
+ *   gate_up_scales  uint8 [E, 2I, H/16] E4M3;  gate_up_scale2 fp32 [E, 2] (gate, up)
+ *                   or NULL (= 1): h[2i] = s_gate * (W x)[2i] + b[2i],
+ *                   h[2i+1] = s_up * (W x)[2i+1] + b[2i+1]
+ *   down_scales     uint8 [E, H, I/16] E4M3;   down_scale2 fp32 [E] or NULL (= 1):
+ *                   y = s_down * (W_d a) + b_d, out = sum_j w_j * y_j
+ * Every other argument, size rule, flag, workspace rule and error as
+ * moe_mxfp4_forward_ex; the workspace size is moe_mxfp4_workspace_size.  scale2
+ * arrays must be 4-byte aligned.  NaN scale bytes set MOE_DEVERR_BAD_SCALE.
+ */
+int moe_nvfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
+                         const int32_t *ids, const float *weights,
+                         const uint8_t *gate_up_blocks, const uint8_t *gate_up_scales,
+                         const float *gate_up_scale2, const float *gate_up_bias,
+                         const uint8_t *down_blocks, const uint8_t *down_scales,
+                         const float *down_scale2, const float *down_bias, float alpha,
+                         float limit, uint16_t *out, uint32_t flags, void *workspace,
+                         size_t workspace_bytes, void *stream);
 
 /* Static English text for a moe_status value. */
 const char *moe_status_string(int status);
@@ -217,7 +266,7 @@ enum {
     MOE_STAGE_GATE_UP = 3, /* gate_up grouped GEMM + bias + clamped SwiGLU */
     MOE_STAGE_DOWN = 4,    /* down grouped GEMM + bias + routing weight   */
     MOE_STAGE_COMBINE = 5, /* per-token sum of the k expert rows          */
-    MOE_STAGE_DEQUANT = 6  /* mxfp4_dequantize                            */
+    MOE_STAGE_DEQUANT = 6  /* mxfp4_dequantize, nvfp4_dequantize          */
 };
 int moe_profile_enable(int on);
 int moe_profile_enable_stages(uint32_t stage_mask);

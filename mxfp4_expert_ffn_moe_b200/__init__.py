@@ -21,6 +21,7 @@ __all__ = [
     "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_enable_stages",
     "moe_profile_read",
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
+    "nvfp4_dequantize", "moe_nvfp4_forward_ex",
 ]
 
 MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -34,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
     "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
+    "nvfp4_dequantize", "moe_nvfp4_forward_ex",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -82,6 +84,12 @@ def load_library():
     lib.moe_profile_enable.restype = i32
     lib.moe_profile_enable_stages.argtypes = [ctypes.c_uint32]
     lib.moe_profile_enable_stages.restype = i32
+    lib.nvfp4_dequantize.argtypes = [p, p, p, p, i64, i64, i64, p]
+    lib.nvfp4_dequantize.restype = i32
+    nv_fwd = [p, i64, i64, i64, i64, i32, p, p, p, p, p, p, p, p, p, p, ctypes.c_float,
+              ctypes.c_float, p, ctypes.c_uint32, p, ctypes.c_size_t, p]
+    lib.moe_nvfp4_forward_ex.argtypes = nv_fwd
+    lib.moe_nvfp4_forward_ex.restype = i32
     lib.moe_profile_read.argtypes = [p, p]
     lib.moe_profile_read.restype = i32
     _lib = lib
@@ -194,6 +202,50 @@ def moe_mxfp4_forward_noalloc(x, ids, weights, gate_up_blocks, gate_up_scales, g
                           down_blocks, down_scales, down_bias, alpha, limit, out)
     rc = load_library().moe_mxfp4_forward_noalloc(*args, ctypes.c_uint32(flags), _stream(stream))
     _check("moe_mxfp4_forward_noalloc", rc)
+    return out
+
+
+def nvfp4_dequantize(blocks, scales, scale2=None, out=None, stream=None):
+    """Packed [E, N, K/2] uint8 + E4M3 [E, N, K/16] uint8 (+ fp32 weight_scale_2 [E])
+    -> bf16 [E, N, K]."""
+    import torch
+    E, N, Kh = blocks.shape
+    K = 2 * Kh
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=blocks.device)
+    rc = load_library().nvfp4_dequantize(_dev(blocks, torch.uint8, "blocks"),
+                                         _dev(scales, torch.uint8, "scales"),
+                                         _dev(scale2, torch.float32, "scale2"),
+                                         _dev(out, torch.bfloat16, "out"), E, N, K, _stream(stream))
+    _check("nvfp4_dequantize", rc)
+    return out
+
+
+def moe_nvfp4_forward_ex(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_scale2,
+                         gate_up_bias, down_blocks, down_scales, down_scale2, down_bias,
+                         alpha: float = 1.702, limit: float = 7.0, out=None, flags: int = 0,
+                         workspace=None, stream=None):
+    """The layer over NVFP4 banks: E4M3 scales [E, 2I, H/16] / [E, H, I/16] and fp32
+    weight_scale_2 [E, 2] (gate, up) / [E], each may be None (= 1)."""
+    import torch
+    T, H = x.shape
+    k = ids.shape[1]
+    E, N2, _ = gate_up_blocks.shape
+    I = N2 // 2
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    ws = _dev(workspace, torch.uint8, "workspace")
+    nbytes = 0 if workspace is None else workspace.numel()
+    rc = load_library().moe_nvfp4_forward_ex(
+        _dev(x, torch.bfloat16, "x"), T, H, I, E, k, _dev(ids, torch.int32, "ids"),
+        _dev(weights, torch.float32, "weights"), _dev(gate_up_blocks, torch.uint8, "gate_up_blocks"),
+        _dev(gate_up_scales, torch.uint8, "gate_up_scales"),
+        _dev(gate_up_scale2, torch.float32, "gate_up_scale2"),
+        _dev(gate_up_bias, torch.float32, "gate_up_bias"), _dev(down_blocks, torch.uint8, "down_blocks"),
+        _dev(down_scales, torch.uint8, "down_scales"), _dev(down_scale2, torch.float32, "down_scale2"),
+        _dev(down_bias, torch.float32, "down_bias"), float(alpha), float(limit),
+        _dev(out, torch.bfloat16, "out"), ctypes.c_uint32(flags), ws, nbytes, _stream(stream))
+    _check("moe_nvfp4_forward_ex", rc)
     return out
 
 

@@ -75,4 +75,120 @@ __global__ void __launch_bounds__(256) mxfp4_dequant_kernel(const uint32_t *__re
     }
 }
 
+// ---- NVFP4 ------------------------------------------------------------------
+// NVFP4 expert banks: the same packed E2M1 codes, one E4M3 scale byte per 16
+// elements ([E, N, K/16]; OCP OFP8 v1.0: bias 7, 3 mantissa bits, subnormals
+// m/8 * 2^-6, S.1111.111 = NaN) and one fp32 weight_scale_2 per expert (FreeToken
+// PR #838, review item "NVFP4 down scale vs. down bias").
+
+// fp32 value of an E4M3 byte (exact); NaN for S.1111.111.
+__device__ __forceinline__ float e4m3_byte_value(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u, sign = (b & 0x80u) << 24;
+    if (e == 15u && m == 7u) return __uint_as_float(0x7FC00000u);
+    const float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0x1p-9f;
+    return __uint_as_float(__float_as_uint(mag) | sign);
+}
+
+// Sticky bit for a truncated product p = RZ(v * s) that sits exactly on a bf16 tie:
+// set the last bit when v * s was inexact, so that the bf16 rounding goes up (in
+// magnitude) as the exact product does.  v has at most 6 significant bits, so the
+// exact product has at most 30: the fma residual is exact while |p| >= 2^-118; below
+// that the product is formed in double, where it is exact.
+__device__ __noinline__ uint32_t tie_sticky(float v, float s, uint32_t b) {
+    const float p = __uint_as_float(b);
+    bool inexact;
+    if (fabsf(p) >= 0x1p-118f) {
+        inexact = __fmaf_rn(v, s, -p) != 0.0f;
+    } else {
+        const double d = (double)v * (double)s;
+        inexact = (double)p != d;
+    }
+    return inexact ? (b | 1u) : b;
+}
+
+// v * s (v with at most 6 significant bits, both finite) as an fp32 whose
+// round-to-nearest-even conversion to bf16 equals rounding the exact product once.
+// Truncating to fp32 keeps the product on the same side of every bf16 rounding
+// boundary unless the truncated value lands exactly on a tie (low 16 bits 0x8000),
+// where the sticky bit decides; this is round-to-odd (Boldo and Melquiond,
+// "Emulation of FMA and correctly rounded sums: proved algorithms using rounding to
+// odd", IEEE Trans. Computers 57(4), 2008) applied only where it can matter.
+__device__ __forceinline__ float mul_for_bf16(float v, float s) {
+    const uint32_t b = __float_as_uint(__fmul_rz(v, s));
+    return __uint_as_float((b & 0xFFFFu) == 0x8000u ? tie_sticky(v, s, b) : b);
+}
+
+// Two fp32 values -> bf16x2; NaN as 0x7fc0 (the slow path for non-finite scale2).
+__device__ __forceinline__ uint32_t pack_bf16x2_canon(float lo, float hi) {
+    uint32_t r = pack_bf16x2(lo, hi);
+    if (lo != lo) r = (r & 0xFFFF0000u) | 0x7FC0u;
+    if (hi != hi) r = (r & 0x0000FFFFu) | 0x7FC00000u;
+    return r;
+}
+
+// out[e, n, kk] = bf16(E2M1(code) * E4M3(scale[e, n, kk/16]) * scale2[e]), rounded
+// once from the exact product; scale2 == nullptr means 1.  Grid: x strides over the
+// words of one expert, y over experts, so weight_scale_2 is one load per block.
+// Each thread turns one 32-bit word (eight codes, half a 16-element block) into one
+// 16-byte bf16 chunk.  Paths: scale2 == 1 (products exact, plain conversion),
+// finite scale2 (mul_for_bf16), non-finite scale2 (canonical NaNs); a NaN scale
+// byte makes its whole word NaN and flags the device error word.
+__device__ __forceinline__ uint4 nvfp4_word(uint32_t q, uint32_t sb, const float *lut, float s2, int mode) {
+    if ((sb & 0x7Fu) == 0x7Fu) {
+        raise_device_error(MOE_DEVERR_BAD_SCALE);
+        return make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+    }
+    const float sc = e4m3_byte_value(sb);
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float a = lut[(q >> (8 * j)) & 15u] * sc;          // exact: <= 6 significant bits
+        float b = lut[(q >> (8 * j + 4)) & 15u] * sc;
+        if (mode == 0) {
+            o[j] = pack_bf16x2(a, b);
+        } else if (mode == 1) {
+            o[j] = pack_bf16x2(mul_for_bf16(a, s2), mul_for_bf16(b, s2));
+        } else {
+            o[j] = pack_bf16x2_canon(a * s2, b * s2);      // inf / NaN scale2: no rounding left
+        }
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(256) nvfp4_dequant_kernel(const uint32_t *__restrict__ packed,
+                                                            const uint8_t *__restrict__ scales,
+                                                            const float *__restrict__ scale2,
+                                                            uint4 *__restrict__ out,
+                                                            int64_t words_per_expert, int64_t E) {
+    __shared__ float lut[16];
+    if (threadIdx.x < 16) {
+        const uint32_t c = threadIdx.x, e = (c >> 1) & 3u, m = c & 1u;
+        float mag = (e == 0u) ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, (int)e - 1);
+        lut[c] = (c & 8u) ? -mag : mag;
+    }
+    __syncthreads();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t e = blockIdx.y; e < E; e += gridDim.y) {
+        const float s2 = scale2 ? __ldg(scale2 + e) : 1.0f;
+        const int mode = s2 == 1.0f ? 0 : (isfinite(s2) ? 1 : 2);   // uniform over the block
+        const uint32_t *src = packed + e * words_per_expert;
+        const uint8_t *sc_e = scales + e * (words_per_expert >> 1);   // 2 words per 16-element block
+        uint4 *dst = out + e * words_per_expert;
+        constexpr int U = 4;
+        int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+        for (; w + (U - 1) * stride < words_per_expert; w += U * stride) {
+            uint32_t word[U], sb[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                word[u] = __ldg(src + w + u * stride);
+                sb[u] = __ldg(sc_e + ((w + u * stride) >> 1));
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) __stcs(dst + w + u * stride, nvfp4_word(word[u], sb[u], lut, s2, mode));
+        }
+        for (; w < words_per_expert; w += stride)
+            __stcs(dst + w, nvfp4_word(__ldg(src + w), __ldg(sc_e + (w >> 1)), lut, s2, mode));
+    }
+}
+
 }  // namespace moe

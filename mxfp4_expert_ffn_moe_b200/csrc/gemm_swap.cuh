@@ -15,6 +15,12 @@
 // FreeToken PR #838: gate_up bias before the gated activation, down bias before
 // the routing weight, sum w*(y + b).)
 //
+// NVFP4 experts (kNv): the same codes with one E4M3 scale per 16 elements decode to
+// E2M1 * E4M3 (exact in bf16: at most 6 significant bits), and the per-expert fp32
+// weight_scale_2 s multiplies the accumulator before the bias, h = s*acc + b and
+// y = s*acc + b, with one s for the gate rows and one for the up rows of gate_up
+// (FreeToken PR #838, review item "NVFP4 down scale vs. down bias": sum w*(s*y + b)).
+//
 // Why weights on M: one tcgen05.mma 128 x TOK x 16 applies every decoded weight
 // element to TOK token rows, so the in-smem decode work per MAC is 1/TOK (1/256 for
 // prefill tiles), and a tile's token count sets the MMA's N, so small decode
@@ -103,8 +109,9 @@ struct Params {
     const int32_t *counts;        // [E]
     const int32_t *offsets;       // [E + 1]
     const int32_t *tile_offsets;  // [E + 1] in TOK-row token tiles
-    const uint8_t *wscales;       // [E, N, K/32]
+    const uint8_t *wscales;       // E8M0 [E, N, K/32] (MXFP4) or E4M3 [E, N, K/16] (NVFP4)
     const float *bias;            // [E, N] or null
+    const float *scale2;          // NVFP4 weight_scale_2: gate_up [E, 2] (gate, up), down [E]; or null
     int E, N, K;
     // gate_up epilogue
     uint16_t *act;                // [rows, N/2] bf16
@@ -164,7 +171,23 @@ __device__ __forceinline__ void e2m1x8_to_bf16_rep(uint32_t q, uint32_t &r0, uin
     r3 = (ptx::prmt(lo, hi, 0x8783u) * 0x1040u) & 0x81C081C0u;
 }
 
-template <class Cfg, bool kGateUp>
+// An E4M3 scale byte as a bf16 pair (exact: 4 significant bits, exponents within
+// bf16's normal range); S.1111.111 is NaN and flags the device error word.
+__device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
+    const uint32_t e = (b >> 3) & 15u, m = b & 7u, sign = (b & 0x80u) << 8;
+    uint32_t h;
+    if (e == 15u && m == 7u) {
+        raise_device_error(MOE_DEVERR_BAD_SCALE);
+        h = 0x7FC0u;
+    } else if (e) {
+        h = sign | ((e + 120u) << 7) | (m << 4);
+    } else {
+        h = sign | (__float_as_uint((float)m * 0x1p-9f) >> 16);   // subnormal m/8 * 2^-6
+    }
+    return h * 0x10001u;
+}
+
+template <class Cfg, bool kGateUp, bool kNv = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_mxfp4_swap_kernel(const __grid_constant__ CUtensorMap tmap_x,
                               const __grid_constant__ CUtensorMap tmap_w, const Params p) {
@@ -303,6 +326,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = r < t.mrows;
             const int n = t.m0 + r;                             // output feature of this thread
             const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
+            // NVFP4 weight_scale_2 of this row (gate rows are even), applied before the bias;
+            // the down projection's is one per expert and is loaded per chunk below
+            const float rs = (kNv && kGateUp && p.scale2 && row_ok) ? __ldg(p.scale2 + 2 * t.e + (n & 1)) : 1.0f;
             // down: lane i holds the pair index and routing weight of token 32 j + i
             int pairs[TOK / 32];
             float wts[TOK / 32];
@@ -315,9 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+                const uint32_t taddr = tmem_base + b * Cfg::ACC_STRIDE + c0 + ((uint32_t)(q * 32) << 16);
                 uint32_t v[32];
-                ptx::tmem_ld_32x32b_x32(tmem_base + b * Cfg::ACC_STRIDE + c0 + ((uint32_t)(q * 32) << 16), v);
-                ptx::tmem_ld_wait();
+                if (kGateUp || !kNv) {
+                    ptx::tmem_ld_32x32b_x32(taddr, v);
+                    ptx::tmem_ld_wait();
+                }
                 const int nvalid = min(32, t.ntok - c0);
                 if (kGateUp) {
                     // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
@@ -330,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + 4096 * q);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float lo_v = __uint_as_float(v[i]), hi_v = __uint_as_float(v[16 + i]);
+                        const float lo_v = rs * __uint_as_float(v[i]), hi_v = rs * __uint_as_float(v[16 + i]);
                         const float mine = odd ? hi_v : lo_v;
                         const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? lo_v : hi_v, 1);
                         const float gate = (odd ? other : mine) + bg;
@@ -355,10 +384,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
                     // so that each pair's row segment leaves as 16-byte stores
                     float *stg = reinterpret_cast<float *>(gbase + Cfg::OFF_EPI + 4096 * q);
+                    if constexpr (kNv) {
+                        // w * (s * acc + bias), s the expert's down weight_scale_2; the
+                        // accumulator comes in two 16-column pieces (register budget)
+                        const float ds = p.scale2 ? __ldg(p.scale2 + t.e) : 1.0f;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], i);
-                        stg[i * 32 + lane] = wi * (__uint_as_float(v[i]) + bias);
+                        for (int hf = 0; hf < 2; ++hf) {
+                            uint32_t u[16];
+                            ptx::tmem_ld_32x32b_x16(taddr + 16u * hf, u);
+                            ptx::tmem_ld_wait();
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], 16 * hf + i);
+                                stg[(16 * hf + i) * 32 + lane] = wi * fmaf(ds, __uint_as_float(u[i]), bias);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], i);
+                            stg[i * 32 + lane] = wi * (__uint_as_float(v[i]) + bias);
+                        }
                     }
                     __syncwarp();
                     if (32 * q < t.mrows) {                      // warp-uniform
@@ -390,6 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // E2M1 * 2^(s-127) exactly; the result goes to the 128-byte swizzled
         // K-major layout the MMA reads.  The E8M0 bytes a thread needs for its
         // group's next step are loaded from global memory one step ahead.
+        // NVFP4: a block's two E4M3 bytes (one per 16 elements) come as one 16-bit
+        // load; the codes are multiplied by 2^126 (exact E2M1) and then by the
+        // E4M3 scale of their half as a bf16 (exact products).
         const int ct = threadIdx.x - 32 * kFirstConvWarp;
         const int grp = ct / kGroupThreads;
         const int gt = ct % kGroupThreads;                    // thread within its group
@@ -404,14 +453,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int blkid = gt + bi * kGroupThreads;
                 const int row = blkid >> 1;
                 rok[bi] = row < t.mrows;
-                srow[bi] = p.wscales + ((int64_t)t.e * p.N + t.m0 + (rok[bi] ? row : 0)) * kblocks + (blkid & 1);
+                srow[bi] = kNv ? p.wscales + ((int64_t)t.e * p.N + t.m0 + (rok[bi] ? row : 0)) * (2 * kblocks) +
+                                     2 * (blkid & 1)
+                               : p.wscales + ((int64_t)t.e * p.N + t.m0 + (rok[bi] ? row : 0)) * kblocks + (blkid & 1);
             }
+            // scale bits of block bi at step kbi (a block past the tile's rows reads 1.0)
+            constexpr uint32_t kOne = kNv ? 0x3838u : 127u;
+            auto load_sc = [&](int bi, int kbi) -> uint32_t {
+                if constexpr (kNv)
+                    return (uint32_t)__ldg(reinterpret_cast<const unsigned short *>(srow[bi] + 4 * kbi));
+                else
+                    return (uint32_t)__ldg(srow[bi] + 2 * kbi);
+            };
             // first step of this tile that belongs to this group
             int kb = (int)((grp - (int)(it % kConvGroups) + kConvGroups) % kConvGroups);
             uint32_t nxt[kBlocksPerThread];
 #pragma unroll
             for (int bi = 0; bi < kBlocksPerThread; ++bi)
-                nxt[bi] = (rok[bi] && kb < k_iters) ? (uint32_t)__ldg(srow[bi] + 2 * kb) : 127u;
+                nxt[bi] = (rok[bi] && kb < k_iters) ? load_sc(bi, kb) : kOne;
             for (; kb < k_iters; kb += kConvGroups) {
                 const uint32_t gi = it + (uint32_t)kb;         // global step index
                 const int c = gi % S, ps = gi % PS;
@@ -419,8 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int bi = 0; bi < kBlocksPerThread; ++bi) {
                     cur[bi] = nxt[bi];
-                    nxt[bi] = (rok[bi] && kb + kConvGroups < k_iters)
-                                  ? (uint32_t)__ldg(srow[bi] + 2 * (kb + kConvGroups)) : 127u;
+                    nxt[bi] = (rok[bi] && kb + kConvGroups < k_iters) ? load_sc(bi, kb + kConvGroups) : kOne;
                 }
                 if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (gi / PS) & 1u)))) break;
                 uint4 q4[kBlocksPerThread];
@@ -435,8 +493,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int blkid = gt + bi * kGroupThreads;    // 0 .. 255 within the step
                     const int row = blkid >> 1, blk = blkid & 1;
                     const uint32_t sc = cur[bi];
-                    uint32_t m1, m2 = 0;
-                    if (sc == 255u) {
+                    uint32_t m1, m2 = 0, m2b = 0;   // m2: words 0-1 (first 16 elements), m2b: words 2-3
+                    if (kNv) {
+                        m1 = 0x7E807E80u;
+                        m2 = e4m3_to_bf16x2(sc & 0xFFu);
+                        m2b = e4m3_to_bf16x2(sc >> 8);
+                    } else if (sc == 255u) {
                         raise_device_error(MOE_DEVERR_BAD_SCALE);
                         m1 = 0x7FC07FC0u;
                     } else if (sc <= 128u) {
@@ -445,6 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         m1 = 0x7E807E80u;
                         m2 = (sc << 7) * 0x10001u;
                     }
+                    if (!kNv) m2b = m2;
                     const uint32_t qw[4] = {q4[bi].x, q4[bi].y, q4[bi].z, q4[bi].w};
                     const uint32_t dst_row = wb_stage(c) + row * 128;
                     const uint32_t sw = (uint32_t)(row & 7);
@@ -456,11 +519,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         r1 = ptx::hmul2_bf16(r1, m1);
                         r2 = ptx::hmul2_bf16(r2, m1);
                         r3 = ptx::hmul2_bf16(r3, m1);
-                        if (m2) {
-                            r0 = ptx::hmul2_bf16(r0, m2);
-                            r1 = ptx::hmul2_bf16(r1, m2);
-                            r2 = ptx::hmul2_bf16(r2, m2);
-                            r3 = ptx::hmul2_bf16(r3, m2);
+                        const uint32_t mw = w < 2 ? m2 : m2b;
+                        if (kNv || mw) {
+                            r0 = ptx::hmul2_bf16(r0, mw);
+                            r1 = ptx::hmul2_bf16(r1, mw);
+                            r2 = ptx::hmul2_bf16(r2, mw);
+                            r3 = ptx::hmul2_bf16(r3, mw);
                         }
                         const uint32_t chunk = (uint32_t)(blk * 4 + w);
                         ptx::st_shared_v4(dst_row + ((chunk ^ sw) << 4), r0, r1, r2, r3);

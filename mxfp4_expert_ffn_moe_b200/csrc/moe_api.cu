@@ -223,10 +223,11 @@ int max_smem_optin() {
 }
 
 // Grouped projection: rows of A (expert order, [rows, K] bf16) x packed weights
-// [E, N, K/2] of each row's expert, with the gate_up or the down epilogue.
-template <class Cfg, bool kGateUp>
+// [E, N, K/2] of each row's expert, with the gate_up or the down epilogue; kNv
+// selects NVFP4 scales (E4M3 per 16 elements, weight_scale_2 in scale2).
+template <class Cfg, bool kGateUp, bool kNv>
 int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, const uint8_t *wblocks,
-                        const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
+                        const uint8_t *wscales, const float *scale2, const float *bias, int64_t E, int64_t N,
                         const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
                         uint16_t *act, float alpha, float limit, float *yp,
                         const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
@@ -237,6 +238,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     p.offsets = offsets;
     p.tile_offsets = tile_offsets;
     p.wscales = wscales;
+    p.scale2 = scale2;
     p.bias = bias;
     p.E = (int)E;
     p.N = (int)N;
@@ -250,7 +252,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     p.weight_on_input = woi;
     const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
-    auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp>;
+    auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp, kNv>;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     const int64_t w_tiles = moe::ceil_div(N, moe::swp::BM);
@@ -262,22 +264,24 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
 }
 
 // Both projections with one tile configuration.
-template <class Cfg>
+template <class Cfg, bool kNv>
 int launch_projections(const uint16_t *x_perm, uint16_t *act, float *yp, int64_t P, int64_t H,
                        int64_t I, int64_t E, const uint8_t *gate_up_blocks,
-                       const uint8_t *gate_up_scales, const float *gate_up_bias,
-                       const uint8_t *down_blocks, const uint8_t *down_scales,
+                       const uint8_t *gate_up_scales, const float *gate_up_scale2,
+                       const float *gate_up_bias, const uint8_t *down_blocks,
+                       const uint8_t *down_scales, const float *down_scale2,
                        const float *down_bias, float alpha, float limit, const int32_t *counts,
                        const int32_t *offsets, const int32_t *tile_offsets,
                        const int32_t *sorted_pairs, const float *weights, bool woi, cudaStream_t s) {
-    int rc = launch_grouped_gemm<Cfg, true>(MOE_STAGE_GATE_UP, x_perm, P, H, gate_up_blocks,
-                                            gate_up_scales, gate_up_bias, E, 2 * I, counts, offsets,
-                                            tile_offsets, act, alpha, limit, nullptr, sorted_pairs,
-                                            weights, 0, s);
+    int rc = launch_grouped_gemm<Cfg, true, kNv>(MOE_STAGE_GATE_UP, x_perm, P, H, gate_up_blocks,
+                                                 gate_up_scales, gate_up_scale2, gate_up_bias, E, 2 * I,
+                                                 counts, offsets, tile_offsets, act, alpha, limit, nullptr,
+                                                 sorted_pairs, weights, 0, s);
     if (rc != MOE_OK) return rc;
-    return launch_grouped_gemm<Cfg, false>(MOE_STAGE_DOWN, act, P, I, down_blocks, down_scales,
-                                           down_bias, E, H, counts, offsets, tile_offsets, nullptr,
-                                           alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
+    return launch_grouped_gemm<Cfg, false, kNv>(MOE_STAGE_DOWN, act, P, I, down_blocks, down_scales,
+                                                down_scale2, down_bias, E, H, counts, offsets, tile_offsets,
+                                                nullptr, alpha, limit, yp, sorted_pairs, weights,
+                                                woi ? 1 : 0, s);
 }
 
 // Block-scaled grouped projection: split rows B ([2][P][K] + scale words) x packed
@@ -371,7 +375,10 @@ bool config_fits(int64_t H, int64_t I) {
     return (int)Cfg::smem_bytes((int)(H / 32)) <= optin && (int)Cfg::smem_bytes((int)(I / 32)) <= optin;
 }
 
-TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E) {
+// NVFP4 banks always take the converter kernel: the block-scaled MMA of the decode
+// tiles reads E8M0 scales per 32 elements only.
+TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E, bool nv) {
+    if (nv) return use_decode_tiles(P, E) ? kDecodeSmem : kPrefillSmem;
     if (use_decode_tiles(P, E))
         return (MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) ? kDecodeMxf : kDecodeSmem;
     return (MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) ? kPrefillMxf : kPrefillSmem;
@@ -384,6 +391,109 @@ int config_tok(TileConfig c) {
         case kDecodeMxf: return moe::mxf::DecodeCfg::TOK;
         default: return moe::mxf::PrefillCfg::TOK;
     }
+}
+
+// The whole layer on the caller's stream: permute -> gather (or split) -> gate_up ->
+// down -> combine.  nv: NVFP4 banks (E4M3 scales per 16 elements, weight_scale_2).
+int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
+                  const int32_t *ids, const float *weights, const uint8_t *gate_up_blocks,
+                  const uint8_t *gate_up_scales, const float *gate_up_scale2, const float *gate_up_bias,
+                  const uint8_t *down_blocks, const uint8_t *down_scales, const float *down_scale2,
+                  const float *down_bias, float alpha, float limit, uint16_t *out, uint32_t flags,
+                  void *workspace, size_t workspace_bytes, void *stream) {
+    if (!x || !ids || !weights || !gate_up_blocks || !gate_up_scales || !down_blocks ||
+        !down_scales || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!forward_sizes_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
+    if (flags & ~MOE_FLAG_WEIGHT_ON_INPUT) return MOE_ERR_INVALID_ARG;
+    const bool woi = (flags & MOE_FLAG_WEIGHT_ON_INPUT) != 0;
+    if (woi && (gate_up_bias || down_bias)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gate_up_blocks, 16) ||
+        !aligned(down_blocks, 16) || !aligned(gate_up_scales, 16) || !aligned(down_scales, 16) ||
+        !aligned(ids, 4) || !aligned(weights, 4) ||
+        !aligned(gate_up_bias, 4) || !aligned(down_bias, 4) ||
+        !aligned(gate_up_scale2, 4) || !aligned(down_scale2, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, kAlign)) return MOE_ERR_INVALID_ARG;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    const Workspace L = workspace_layout(T, H, I, E, k);
+    bool owned = false;
+    if (!workspace) {
+        if (cudaMallocAsync(&workspace, L.total, s) != cudaSuccess) {
+            cudaGetLastError();
+            return MOE_ERR_NO_MEMORY;
+        }
+        owned = true;
+    } else if (workspace_bytes < L.total) {
+        return MOE_ERR_NO_MEMORY;
+    }
+    char *ws = static_cast<char *>(workspace);
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    int32_t *tile_offsets = reinterpret_cast<int32_t *>(ws + L.tile_offsets);
+    int32_t *sorted_pairs = reinterpret_cast<int32_t *>(ws + L.sorted_pairs);
+    uint16_t *x_perm = reinterpret_cast<uint16_t *>(ws + L.x_perm);
+    uint16_t *act = reinterpret_cast<uint16_t *>(ws + L.act);
+    float *yp = reinterpret_cast<float *>(ws + L.yp);
+
+    const int64_t P = T * k;
+    const TileConfig cfg = pick_config(P, H, I, E, nv);
+    int rc = MOE_OK;
+    do {
+        {
+            const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
+            StageScope sp(MOE_STAGE_PERMUTE, s);
+            launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P,
+                       (int)E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs);
+        }
+        if ((rc = launch_check()) != MOE_OK) break;
+        const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
+        if (mxf) {
+            uint8_t *xq = reinterpret_cast<uint8_t *>(x_perm);
+            uint8_t *actq = reinterpret_cast<uint8_t *>(act);
+#define MOE_MXF_LAYER(C)                                                                          \
+    launch_mxf_layer<C>(x, weights, sorted_pairs, xq, actq, yp, P, H, I, E, k, gate_up_blocks,           \
+                        gate_up_scales, gate_up_bias, down_blocks, down_scales, down_bias, alpha,    \
+                        limit, counts, offsets, tile_offsets, woi, s)
+            rc = cfg == kDecodeMxf ? MOE_MXF_LAYER(moe::mxf::DecodeCfg) : MOE_MXF_LAYER(moe::mxf::PrefillCfg);
+#undef MOE_MXF_LAYER
+            if (rc != MOE_OK) break;
+        } else {
+            {
+                const int64_t gather_grid =
+                    moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
+                StageScope sg(MOE_STAGE_GATHER, s);
+                launch_pdl(moe::gather_rows_kernel, dim3((unsigned)gather_grid), dim3(256), 0, s, x, weights,
+                           sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
+            }
+            if ((rc = launch_check()) != MOE_OK) break;
+#define MOE_PROJECTIONS(C, NV)                                                                    \
+    launch_projections<C, NV>(x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales,           \
+                              gate_up_scale2, gate_up_bias, down_blocks, down_scales, down_scale2,   \
+                              down_bias, alpha, limit, counts, offsets, tile_offsets, sorted_pairs,  \
+                              weights, woi, s)
+            if (nv)
+                rc = cfg == kDecodeSmem ? MOE_PROJECTIONS(moe::swp::DecodeCfg, true)
+                                        : MOE_PROJECTIONS(moe::swp::PrefillCfg, true);
+            else
+                rc = cfg == kDecodeSmem ? MOE_PROJECTIONS(moe::swp::DecodeCfg, false)
+                                        : MOE_PROJECTIONS(moe::swp::PrefillCfg, false);
+#undef MOE_PROJECTIONS
+        }
+        if (rc != MOE_OK) break;
+        {
+            const int64_t n4 = T * (H / 4);
+            const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;
+            StageScope sc(MOE_STAGE_COMBINE, s);
+            launch_pdl(moe::combine_rows_kernel, dim3((unsigned)cgrid), dim3(256), 0, s, yp, ids, T, k, (int)E, H,
+                       out);
+        }
+        rc = launch_check();
+    } while (0);
+
+    if (owned && cudaFreeAsync(workspace, s) != cudaSuccess && rc == MOE_OK) rc = MOE_ERR_CUDA;
+    return rc;
 }
 
 }  // namespace
@@ -415,6 +525,32 @@ int mxfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out
     StageScope scope(MOE_STAGE_DEQUANT, (cudaStream_t)stream);
     moe::mxfp4_dequant_kernel<<<grid, threads, 0, (cudaStream_t)stream>>>(
         reinterpret_cast<const uint32_t *>(blocks), scales, reinterpret_cast<uint4 *>(out), n_words);
+    return launch_check();
+}
+
+int nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2, uint16_t *out,
+                     int64_t E, int64_t N, int64_t K, void *stream) {
+    if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || N < 1 || K < 16 || K % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(blocks, 16) || !aligned(out, 16) || !aligned(scale2, 4)) return MOE_ERR_INVALID_ARG;
+    const int64_t words_per_expert = N * (K / 8);
+    const int threads = 256;
+    // one wave: as many blocks as the SMs hold at once, spread over the experts
+    static int per_sm = 0;
+    if (per_sm == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::nvfp4_dequant_kernel, threads, 0) !=
+             cudaSuccess || per_sm < 1))
+        per_sm = 4;
+    const int64_t target = (int64_t)sm_count() * per_sm;
+    const int64_t gy = E < 65535 ? E : 65535;
+    int64_t gx = target / gy;
+    const int64_t need_x = moe::ceil_div(words_per_expert, threads);
+    if (gx > need_x) gx = need_x;
+    if (gx < 1) gx = 1;
+    StageScope scope(MOE_STAGE_DEQUANT, (cudaStream_t)stream);
+    moe::nvfp4_dequant_kernel<<<dim3((unsigned)gx, (unsigned)gy), threads, 0, (cudaStream_t)stream>>>(
+        reinterpret_cast<const uint32_t *>(blocks), scales, scale2, reinterpret_cast<uint4 *>(out),
+        words_per_expert, E);
     return launch_check();
 }
 
@@ -458,92 +594,22 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                          const uint8_t *down_scales, const float *down_bias, float alpha,
                          float limit, uint16_t *out, uint32_t flags, void *workspace,
                          size_t workspace_bytes, void *stream) {
-    if (!x || !ids || !weights || !gate_up_blocks || !gate_up_scales || !down_blocks ||
-        !down_scales || !out)
-        return MOE_ERR_INVALID_ARG;
-    if (!forward_sizes_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
-    if (flags & ~MOE_FLAG_WEIGHT_ON_INPUT) return MOE_ERR_INVALID_ARG;
-    const bool woi = (flags & MOE_FLAG_WEIGHT_ON_INPUT) != 0;
-    if (woi && (gate_up_bias || down_bias)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gate_up_blocks, 16) ||
-        !aligned(down_blocks, 16) || !aligned(gate_up_scales, 16) || !aligned(down_scales, 16) ||
-        !aligned(ids, 4) || !aligned(weights, 4) ||
-        !aligned(gate_up_bias, 4) || !aligned(down_bias, 4))
-        return MOE_ERR_INVALID_ARG;
-    if (workspace && !aligned(workspace, kAlign)) return MOE_ERR_INVALID_ARG;
+    return forward_layer(false, x, T, H, I, E, k, ids, weights, gate_up_blocks, gate_up_scales, nullptr,
+                         gate_up_bias, down_blocks, down_scales, nullptr, down_bias, alpha, limit, out,
+                         flags, workspace, workspace_bytes, stream);
+}
 
-    cudaStream_t s = (cudaStream_t)stream;
-    const Workspace L = workspace_layout(T, H, I, E, k);
-    bool owned = false;
-    if (!workspace) {
-        if (cudaMallocAsync(&workspace, L.total, s) != cudaSuccess) {
-            cudaGetLastError();
-            return MOE_ERR_NO_MEMORY;
-        }
-        owned = true;
-    } else if (workspace_bytes < L.total) {
-        return MOE_ERR_NO_MEMORY;
-    }
-    char *ws = static_cast<char *>(workspace);
-    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
-    int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
-    int32_t *tile_offsets = reinterpret_cast<int32_t *>(ws + L.tile_offsets);
-    int32_t *sorted_pairs = reinterpret_cast<int32_t *>(ws + L.sorted_pairs);
-    uint16_t *x_perm = reinterpret_cast<uint16_t *>(ws + L.x_perm);
-    uint16_t *act = reinterpret_cast<uint16_t *>(ws + L.act);
-    float *yp = reinterpret_cast<float *>(ws + L.yp);
-
-    const int64_t P = T * k;
-    const TileConfig cfg = pick_config(P, H, I, E);
-    int rc = MOE_OK;
-    do {
-        {
-            const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
-            StageScope sp(MOE_STAGE_PERMUTE, s);
-            launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P,
-                       (int)E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs);
-        }
-        if ((rc = launch_check()) != MOE_OK) break;
-        const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
-        if (mxf) {
-            uint8_t *xq = reinterpret_cast<uint8_t *>(x_perm);
-            uint8_t *actq = reinterpret_cast<uint8_t *>(act);
-#define MOE_MXF_LAYER(C)                                                                          \
-    launch_mxf_layer<C>(x, weights, sorted_pairs, xq, actq, yp, P, H, I, E, k, gate_up_blocks,           \
-                        gate_up_scales, gate_up_bias, down_blocks, down_scales, down_bias, alpha,    \
-                        limit, counts, offsets, tile_offsets, woi, s)
-            rc = cfg == kDecodeMxf ? MOE_MXF_LAYER(moe::mxf::DecodeCfg) : MOE_MXF_LAYER(moe::mxf::PrefillCfg);
-#undef MOE_MXF_LAYER
-            if (rc != MOE_OK) break;
-        } else {
-            {
-                const int64_t gather_grid =
-                    moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
-                StageScope sg(MOE_STAGE_GATHER, s);
-                launch_pdl(moe::gather_rows_kernel, dim3((unsigned)gather_grid), dim3(256), 0, s, x, weights,
-                           sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
-            }
-            if ((rc = launch_check()) != MOE_OK) break;
-#define MOE_PROJECTIONS(C)                                                                       \
-    launch_projections<C>(x_perm, act, yp, P, H, I, E, gate_up_blocks, gate_up_scales, gate_up_bias, \
-                          down_blocks, down_scales, down_bias, alpha, limit, counts, offsets,         \
-                          tile_offsets, sorted_pairs, weights, woi, s)
-            rc = cfg == kDecodeSmem ? MOE_PROJECTIONS(moe::swp::DecodeCfg) : MOE_PROJECTIONS(moe::swp::PrefillCfg);
-#undef MOE_PROJECTIONS
-        }
-        if (rc != MOE_OK) break;
-        {
-            const int64_t n4 = T * (H / 4);
-            const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;
-            StageScope sc(MOE_STAGE_COMBINE, s);
-            launch_pdl(moe::combine_rows_kernel, dim3((unsigned)cgrid), dim3(256), 0, s, yp, ids, T, k, (int)E, H,
-                       out);
-        }
-        rc = launch_check();
-    } while (0);
-
-    if (owned && cudaFreeAsync(workspace, s) != cudaSuccess && rc == MOE_OK) rc = MOE_ERR_CUDA;
-    return rc;
+int moe_nvfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
+                         const int32_t *ids, const float *weights,
+                         const uint8_t *gate_up_blocks, const uint8_t *gate_up_scales,
+                         const float *gate_up_scale2, const float *gate_up_bias,
+                         const uint8_t *down_blocks, const uint8_t *down_scales,
+                         const float *down_scale2, const float *down_bias, float alpha,
+                         float limit, uint16_t *out, uint32_t flags, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    return forward_layer(true, x, T, H, I, E, k, ids, weights, gate_up_blocks, gate_up_scales,
+                         gate_up_scale2, gate_up_bias, down_blocks, down_scales, down_scale2, down_bias,
+                         alpha, limit, out, flags, workspace, workspace_bytes, stream);
 }
 
 int moe_mxfp4_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,

@@ -25,6 +25,36 @@ def layer_to_device(layer):
     )
 
 
+def nvfp4_layer_to_device(layer):
+    dev = layer_to_device(layer)
+    dev["gu_scale2"] = to_dev(layer.gate_up.scale2)
+    dev["d_scale2"] = to_dev(layer.down.scale2)
+    return dev
+
+
+def run_nvfp4_forward(moe, dev, ids, w, layer, flags=None, workspace=None):
+    import torch
+    ids_d = ids if isinstance(ids, torch.Tensor) else to_dev(ids.astype(np.int32))
+    w_d = w if isinstance(w, torch.Tensor) else to_dev(w.astype(np.float32))
+    if flags is None:
+        flags = moe.MOE_FLAG_WEIGHT_ON_INPUT if layer.weight_on_input else 0
+    out = moe.moe_nvfp4_forward_ex(dev["x"], ids_d, w_d, dev["gu_blocks"], dev["gu_scales"],
+                                   dev["gu_scale2"], dev["gu_bias"], dev["d_blocks"], dev["d_scales"],
+                                   dev["d_scale2"], dev["d_bias"], alpha=layer.alpha, limit=layer.limit,
+                                   flags=flags, workspace=workspace)
+    torch.cuda.synchronize()
+    return out
+
+
+def oracle_nvfp4_forward(oracle, layer, ids, w, tokens=None, envelope=False):
+    return oracle.nvfp4_forward_tokens(layer.x_bits, ids, w, layer.gate_up.blocks, layer.gate_up.scales,
+                                       layer.gate_up.scale2, layer.gate_up_bias, layer.down.blocks,
+                                       layer.down.scales, layer.down.scale2, layer.down_bias,
+                                       alpha=layer.alpha, limit=layer.limit,
+                                       weight_on_input=layer.weight_on_input, tokens=tokens,
+                                       envelope=envelope)
+
+
 def bf16_tensor_to_f64(t):
     import torch
     bits = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
