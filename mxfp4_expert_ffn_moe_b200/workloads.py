@@ -169,5 +169,34 @@ WORKLOADS = {
 }
 
 
+@dataclass
+class Router:
+    """Router linear layer inputs: x bf16 bits [T, H], W_r bf16 bits [E, H], b_r fp32 [E]."""
+    x_bits: np.ndarray
+    w_bits: np.ndarray
+    bias: Optional[np.ndarray]
+    k: int
+
+
+def make_router(T: int, H: int, E: int, k: int, seed: int = 0, bias: bool = True) -> Router:
+    """x ~ N(0, 1), W_r ~ N(0, 1/H) (logits of unit scale), b_r ~ N(0, 0.1^2); in that order."""
+    rng = np.random.default_rng(seed)
+    x_bits = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    w_bits = f32_to_bf16_bits((rng.standard_normal((E, H)) / np.sqrt(H)).astype(np.float32))
+    b = (0.1 * rng.standard_normal(E)).astype(np.float32)
+    return Router(x_bits, w_bits, b if bias else None, k)
+
+
+ROUTERS = {
+    "router_20b_T4096": dict(T=4096, H=2880, E=32, k=4),
+    "router_20b_T8": dict(T=8, H=2880, E=32, k=4),
+    "router_120b_T8192": dict(T=8192, H=2880, E=128, k=4),
+}
+
+
+def router_workload(name: str, seed: int = 0) -> Router:
+    return make_router(seed=seed, **ROUTERS[name])
+
+
 def workload(name: str, seed: int = 0) -> MoELayer:
     return make_layer(seed=seed, name=name, **WORKLOADS[name])

@@ -13,6 +13,8 @@ What each entry point follows is cited in ``moe_oracle.c``; in short:
   E8M0 byte validity); OCP MX v1.0 for the E2M1 and E8M0 element definitions.
 * ``route``       -- top-k over router logits then softmax over the k chosen
   (transformers PR #49431: the MXFP4 experts take routing ids + weights).
+* ``router_logits`` -- the router linear layer before it, x . W_r^T + b_r (FreeToken
+  PR #838: the gpt-oss router is mlp.router, with a bias).
 * ``forward_tokens`` / ``forward_grouped`` -- FreeToken PR #838 "feat(gguf): serve
   gpt-oss gguf checkpoints on gpt_oss", review items on the down bias and on
   apply_router_weight_on_input, and "What it does" (alpha 1.702, limit 7, bias roles).
@@ -102,6 +104,8 @@ def _load():
                                                     p, p, p, p, p, p, p, p, ctypes.c_double,
                                                     ctypes.c_double, ctypes.c_int, p, i64, p, p,
                                                     ctypes.c_int]
+        lib.oracle_router_logits.restype = None
+        lib.oracle_router_logits.argtypes = [p, p, p, i64, i64, i64, p]
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -202,6 +206,20 @@ def forward_grouped(x_bits, ids, weights, gu_blocks, gu_scales, gu_bias, d_block
         FLAG_WEIGHT_ON_INPUT if weight_on_input else 0, _ptr(out))
     if rc != 0:
         raise MemoryError("oracle_forward_grouped: allocation failed")
+    return out
+
+
+def router_logits(x_bits, w_bits, bias=None) -> np.ndarray:
+    """Router linear layer: bf16 x [T,H] and W_r [E,H] (bits), fp32 bias [E] or None
+    -> float64 logits [T,E]."""
+    x_bits = _c(x_bits, np.uint16)
+    w_bits = _c(w_bits, np.uint16)
+    T, H = x_bits.shape
+    E = w_bits.shape[0]
+    assert w_bits.shape[1] == H
+    out = np.empty((T, E), dtype=np.float64)
+    _load().oracle_router_logits(_ptr(x_bits), _ptr(w_bits), _ptr(_c(bias, np.float32)), T, H, E,
+                                 _ptr(out))
     return out
 
 

@@ -26,6 +26,8 @@
  *   [P4] transformers PR #49431, "Restore GPT-OSS's router-masked expert-parallel
  *        plan": the MXFP4 experts consume routing data (ids and weights), not a
  *        dispatch of expert ids.
+ *   [P3'] FreeToken PR #838, section "What it does" and the loader notes: the gpt-oss
+ *        router is the module mlp.router, whose bias loads with the dense state dict.
  *   [MX] OCP Microscaling Formats (MX) v1.0: FP4 E2M1 element (1 sign, 2 exponent
  *        bits with bias 1, 1 mantissa bit, no inf/NaN) and E8M0 scale (2^(b-127),
  *        0xff = NaN).
@@ -53,6 +55,8 @@
  *       of the per-expert triple the review indexes, down being index 2).
  *   R7  the standalone NVFP4 dequant returns bf16 rounded once (nearest, ties to even)
  *       from the exact product E2M1 * E4M3 * weight_scale_2.
+ *   R8  the router is a linear layer with bias: logits[t, e] = x[t] . W_r[e] + b_r[e],
+ *       x and W_r bf16 [T, H] / [E, H], b_r fp32 [E] (a bf16 bias converts exactly).
  *
  * Function that is not pinned by anything outside itself: none -- every entry
  * point is checked against hand-written values, closed forms, invariants or a
@@ -275,6 +279,20 @@ void oracle_route(const float *logits, int64_t T, int64_t E, int k,
     }
     free(ex);
     free(taken);
+}
+
+/* ---- router logits (reading R8; [P3'] mlp.router with its bias) -------------- */
+/* out[t, e] = sum_c x[t, c] * W[e, c] + b[e] in double; x, W bf16 bits; b may be NULL. */
+void oracle_router_logits(const uint16_t *x, const uint16_t *w, const float *b, int64_t T,
+                          int64_t H, int64_t E, double *out)
+{
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < H; ++c)
+                acc += oracle_bf16_to_double(x[t * H + c]) * oracle_bf16_to_double(w[e * H + c]);
+            out[t * E + e] = acc + (b ? (double)b[e] : 0.0);
+        }
 }
 
 /* ---- clamped SwiGLU (reading R4; constants from [P3] What it does) ---------- */
