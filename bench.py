@@ -358,6 +358,30 @@ def extra_measurements(device, stream, peaks):
     del banks
     torch.cuda.empty_cache()
 
+    # router linear layer fused with routing (tensor-core GEMM + top-k epilogue)
+    from mxfp4_expert_ffn_moe_b200.workloads import router_workload
+    for name in ("router_20b_T8", "router_20b_T4096", "router_120b_T8192"):
+        r = router_workload(name)
+        T, H = r.x_bits.shape
+        E = r.w_bits.shape[0]
+        x = torch.from_numpy(r.x_bits).view(torch.bfloat16).to(device)
+        w = torch.from_numpy(r.w_bits).view(torch.bfloat16).to(device)
+        b = torch.from_numpy(r.bias).to(device)
+        ids = torch.empty((T, r.k), dtype=torch.int32, device=device)
+        wt = torch.empty((T, r.k), dtype=torch.float32, device=device)
+
+        def rr():
+            moe.moe_router_route(x, w, b, r.k, ids=ids, weights=wt)
+
+        for _ in range(3):
+            rr()
+        ms = time_steps(rr, 20, stream, flush) / 20
+        nbytes = 2 * T * H + 2 * E * H + 4 * E + 8 * T * r.k
+        res[name] = {"us": ms * 1e3, "tokens/s": T / (ms * 1e-3), "GB/s": nbytes / (ms * 1e-3) / 1e9,
+                     "TFLOP/s": 2.0 * T * E * H / (ms * 1e-3) / 1e12, "bytes": nbytes}
+        del x, w, b, ids, wt
+    torch.cuda.empty_cache()
+
     for name, steps, do_flush in [("20b_decode_T1", 50, True), ("20b_decode_T8", 50, True),
                                   ("20b_decode_T64", 30, True), ("120b_zipf_T256", 20, True),
                                   ("120b_zipf_T8192", 5, False), ("nvfp4_20b_decode_T8", 50, True),

@@ -102,6 +102,23 @@ int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *
               float *weights, void *stream);
 
 /*
+ * moe_router_route -- the router linear layer fused with moe_route (FreeToken PR #838:
+ * the gpt-oss router is the linear module mlp.router, with a bias):
+ *   logits[t, e] = x[t] . w_router[e] + b_router[e]   (bf16 operands, fp32 accumulate
+ *                                                       on the tensor cores)
+ *   ids, weights  = moe_route of those fp32 logits (same selection rule and softmax)
+ *   x         bf16 [T, H];  w_router bf16 [E, H];  b_router fp32 [E] or NULL (= zero)
+ *   logits    fp32 [T, E] or NULL: when given, receives the logits the routing used
+ *   ids int32 [T, k]; weights fp32 [T, k]
+ * Sizes: T >= 1; H >= 64 and H % 64 == 0; 1 <= E <= 256; 1 <= k <= min(E, 8).  x and
+ * w_router must be 16-byte aligned.  Errors: MOE_ERR_INVALID_ARG for null pointers,
+ * sizes or alignment; MOE_ERR_UNSUPPORTED for E > 256.
+ */
+int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b_router, int64_t T,
+                     int64_t H, int64_t E, int k, float *logits, int32_t *ids, float *weights,
+                     void *stream);
+
+/*
  * moe_mxfp4_forward -- the expert layer, weights on the output
  * (FreeToken PR #838: sum w*(y + b); bias before the routing weight):
  *   x               bf16  [T, H]

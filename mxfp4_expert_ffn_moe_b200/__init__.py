@@ -21,7 +21,7 @@ __all__ = [
     "EXPORTED_SYMBOLS", "PROFILE_STAGES", "moe_profile_enable", "moe_profile_enable_stages",
     "moe_profile_read",
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
-    "nvfp4_dequantize", "moe_nvfp4_forward_ex",
+    "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
 ]
 
 MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -35,7 +35,7 @@ EXPORTED_SYMBOLS = (
     "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
     "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
-    "nvfp4_dequantize", "moe_nvfp4_forward_ex",
+    "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -84,6 +84,8 @@ def load_library():
     lib.moe_profile_enable.restype = i32
     lib.moe_profile_enable_stages.argtypes = [ctypes.c_uint32]
     lib.moe_profile_enable_stages.restype = i32
+    lib.moe_router_route.argtypes = [p, p, p, i64, i64, i64, i32, p, p, p, p]
+    lib.moe_router_route.restype = i32
     lib.nvfp4_dequantize.argtypes = [p, p, p, p, i64, i64, i64, p]
     lib.nvfp4_dequantize.restype = i32
     nv_fwd = [p, i64, i64, i64, i64, i32, p, p, p, p, p, p, p, p, p, p, ctypes.c_float,
@@ -149,6 +151,28 @@ def moe_route(router_logits, k: int, ids=None, weights=None, stream=None):
                                   _stream(stream))
     _check("moe_route", rc)
     return ids, weights
+
+
+def moe_router_route(x, w_router, b_router, k: int, want_logits: bool = False, ids=None,
+                     weights=None, logits=None, stream=None):
+    """Router linear layer + routing: bf16 x [T, H], bf16 w_router [E, H], fp32 b_router
+    [E] or None -> (int32 ids [T, k], fp32 weights [T, k]) and, with want_logits (or a
+    logits tensor given), the fp32 logits [T, E] the routing used."""
+    import torch
+    T, H = x.shape
+    E = w_router.shape[0]
+    if ids is None:
+        ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    if weights is None:
+        weights = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    if logits is None and want_logits:
+        logits = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    rc = load_library().moe_router_route(
+        _dev(x, torch.bfloat16, "x"), _dev(w_router, torch.bfloat16, "w_router"),
+        _dev(b_router, torch.float32, "b_router"), T, H, E, int(k), _dev(logits, torch.float32, "logits"),
+        _dev(ids, torch.int32, "ids"), _dev(weights, torch.float32, "weights"), _stream(stream))
+    _check("moe_router_route", rc)
+    return (ids, weights, logits) if logits is not None else (ids, weights)
 
 
 def _fwd_args(x, ids, weights, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,

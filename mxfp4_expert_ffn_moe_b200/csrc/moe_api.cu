@@ -22,6 +22,7 @@
 #include "permute.cuh"
 #include "split.cuh"
 #include "route.cuh"
+#include "router.cuh"
 
 namespace {
 
@@ -579,6 +580,32 @@ int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *
 #undef MOE_ROUTE_CASE
         default: return MOE_ERR_UNSUPPORTED;
     }
+    return launch_check();
+}
+
+int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b_router, int64_t T,
+                     int64_t H, int64_t E, int k, float *logits, int32_t *ids, float *weights,
+                     void *stream) {
+    if (!x || !w_router || !ids || !weights) return MOE_ERR_INVALID_ARG;
+    if (T < 1 || T > (int64_t)0x7FFFFFFF - moe::rtr::BM) return MOE_ERR_INVALID_ARG;
+    if (H < 64 || H % 64 != 0 || H > (int64_t)0x7FFFFFFF) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID_ARG;
+    if (E > 256) return MOE_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(b_router, 4) || !aligned(logits, 4) ||
+        !aligned(ids, 4) || !aligned(weights, 4))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    CUtensorMap mx, mw;
+    if (!make_act_map(&mx, x, T, H) || !make_act_map(&mw, w_router, E, H)) return MOE_ERR_CUDA;
+    const uint32_t smem = moe::rtr::smem_bytes((int)E);
+    if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(moe::rtr::router_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int64_t grid = moe::ceil_div(T, moe::rtr::BM);
+    StageScope scope(MOE_STAGE_ROUTE, s);
+    launch_pdl(moe::rtr::router_route_kernel, dim3((unsigned)grid), dim3(moe::rtr::kThreads), smem, s, mx, mw,
+               b_router, (int)T, (int)H, (int)E, k, logits, ids, weights);
     return launch_check();
 }
 
