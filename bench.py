@@ -358,6 +358,38 @@ def extra_measurements(device, stream, peaks):
     del banks
     torch.cuda.empty_cache()
 
+    # dequant-on-copy from host memory: the gpt-oss-20b down bank in page-locked host
+    # memory, decoded by the kernel through its device mapping, against a plain
+    # copy-engine transfer of the same packed bytes (the host link's rate)
+    _, dn = make_dequant_bank(seed=0)
+    E, N, K = dn.shape
+    hb = torch.from_numpy(dn.blocks).pin_memory()
+    hs = torch.from_numpy(dn.scales).pin_memory()
+    o = torch.empty((E, N, K), dtype=torch.bfloat16, device=device)
+    db = torch.empty(dn.blocks.shape, dtype=torch.uint8, device=device)
+    ds = torch.empty(dn.scales.shape, dtype=torch.uint8, device=device)
+
+    def from_host():
+        moe.mxfp4_dequantize_from_host(hb, hs, out=o)
+
+    def copy_packed():
+        db.copy_(hb, non_blocking=True)
+        ds.copy_(hs, non_blocking=True)
+
+    for _ in range(2):
+        from_host()
+        copy_packed()
+    ms_h = time_steps(from_host, 5, stream) / 5
+    ms_c = time_steps(copy_packed, 5, stream) / 5
+    packed = dn.blocks.nbytes + dn.scales.nbytes
+    res["dequant_from_host_20b_down"] = {
+        "ms": ms_h, "packed_bytes": packed, "bf16_bytes_written": E * N * K * 2,
+        "host_link_GB/s": packed / (ms_h * 1e-3) / 1e9,
+        "copy_engine_GB/s_same_bytes": packed / (ms_c * 1e-3) / 1e9,
+        "frac_of_copy_engine": ms_c / ms_h}
+    del hb, hs, o, db, ds
+    torch.cuda.empty_cache()
+
     # router linear layer fused with routing (tensor-core GEMM + top-k epilogue)
     from mxfp4_expert_ffn_moe_b200.workloads import router_workload
     for name in ("router_20b_T8", "router_20b_T4096", "router_120b_T8192"):

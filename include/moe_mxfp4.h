@@ -32,7 +32,8 @@
  *
  * Conventions for every call:
  *   - All tensor pointers are caller-owned DEVICE memory on the current CUDA
- *     device, contiguous row-major, never freed or retained by the library.
+ *     device, contiguous row-major, never freed or retained by the library (the
+ *     *_from_host calls take their packed bank in page-locked HOST memory instead).
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *     enqueued on it; no call synchronises the host (except
@@ -88,6 +89,26 @@ typedef enum {
  */
 int mxfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out,
                      int64_t E, int64_t N, int64_t K, void *stream);
+
+/*
+ * mxfp4_dequantize_from_host / nvfp4_dequantize_from_host -- dequant-on-copy from host
+ * memory (MoE-Infinity PR #152, Changes: fetched packed experts are dequantised on
+ * copy).  As mxfp4_dequantize / nvfp4_dequantize, but host_blocks and host_scales are
+ * page-locked HOST memory that the current device can address (cudaHostAlloc /
+ * cudaMallocHost, or a cudaHostRegister'd range; mapped under unified addressing):
+ * the decode kernel reads the packed codes over the host link through the device
+ * mapping and writes bf16 straight into `out` (device memory), so 4.25 (MXFP4) or
+ * 4.5 (NVFP4) bits per weight cross the link instead of 16.  scale2 (NVFP4) is device
+ * memory or NULL.  Both host buffers must hold the whole bank; MOE_ERR_INVALID_ARG
+ * when the first or last byte of either is not such host memory, or for the sizes
+ * and alignment rules of the device-memory calls.  The host memory must stay
+ * allocated and unmodified until the stream has run the call.
+ */
+int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales, uint16_t *out,
+                               int64_t E, int64_t N, int64_t K, void *stream);
+int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales,
+                               const float *scale2, uint16_t *out, int64_t E, int64_t N, int64_t K,
+                               void *stream);
 
 /*
  * moe_route -- top-k routing (transformers PR #49431: the MXFP4 experts consume
@@ -283,7 +304,7 @@ enum {
     MOE_STAGE_GATE_UP = 3, /* gate_up grouped GEMM + bias + clamped SwiGLU */
     MOE_STAGE_DOWN = 4,    /* down grouped GEMM + bias + routing weight   */
     MOE_STAGE_COMBINE = 5, /* per-token sum of the k expert rows          */
-    MOE_STAGE_DEQUANT = 6  /* mxfp4_dequantize, nvfp4_dequantize          */
+    MOE_STAGE_DEQUANT = 6  /* mxfp4_ / nvfp4_dequantize (+ _from_host)   */
 };
 int moe_profile_enable(int on);
 int moe_profile_enable_stages(uint32_t stage_mask);

@@ -22,6 +22,7 @@ __all__ = [
     "moe_profile_read",
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
+    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host",
 ]
 
 MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -36,6 +37,7 @@ EXPORTED_SYMBOLS = (
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
     "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
+    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -86,6 +88,10 @@ def load_library():
     lib.moe_profile_enable_stages.restype = i32
     lib.moe_router_route.argtypes = [p, p, p, i64, i64, i64, i32, p, p, p, p]
     lib.moe_router_route.restype = i32
+    lib.mxfp4_dequantize_from_host.argtypes = [p, p, p, i64, i64, i64, p]
+    lib.mxfp4_dequantize_from_host.restype = i32
+    lib.nvfp4_dequantize_from_host.argtypes = [p, p, p, p, i64, i64, i64, p]
+    lib.nvfp4_dequantize_from_host.restype = i32
     lib.nvfp4_dequantize.argtypes = [p, p, p, p, i64, i64, i64, p]
     lib.nvfp4_dequantize.restype = i32
     nv_fwd = [p, i64, i64, i64, i64, i32, p, p, p, p, p, p, p, p, p, p, ctypes.c_float,
@@ -135,6 +141,43 @@ def mxfp4_dequantize(blocks, scales, out=None, stream=None):
                                          _dev(scales, torch.uint8, "scales"),
                                          _dev(out, torch.bfloat16, "out"), E, N, K, _stream(stream))
     _check("mxfp4_dequantize", rc)
+    return out
+
+
+def _host(t, dtype, name):
+    if not (t.device.type == "cpu" and t.dtype == dtype and t.is_contiguous() and t.is_pinned()):
+        raise ValueError(f"{name}: expected a contiguous page-locked CPU {dtype} tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def mxfp4_dequantize_from_host(blocks, scales, out=None, device=None, stream=None):
+    """Dequant-on-copy: packed [E, N, K/2] + E8M0 [E, N, K/32] in pinned host memory ->
+    bf16 [E, N, K] on the device (the kernel reads the host bank through its mapping)."""
+    import torch
+    E, N, Kh = blocks.shape
+    K = 2 * Kh
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=device or "cuda")
+    rc = load_library().mxfp4_dequantize_from_host(_host(blocks, torch.uint8, "blocks"),
+                                                   _host(scales, torch.uint8, "scales"),
+                                                   _dev(out, torch.bfloat16, "out"), E, N, K, _stream(stream))
+    _check("mxfp4_dequantize_from_host", rc)
+    return out
+
+
+def nvfp4_dequantize_from_host(blocks, scales, scale2=None, out=None, device=None, stream=None):
+    """Dequant-on-copy of an NVFP4 bank in pinned host memory (E4M3 [E, N, K/16]);
+    scale2 is a device fp32 [E] tensor or None."""
+    import torch
+    E, N, Kh = blocks.shape
+    K = 2 * Kh
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=device or "cuda")
+    rc = load_library().nvfp4_dequantize_from_host(_host(blocks, torch.uint8, "blocks"),
+                                                   _host(scales, torch.uint8, "scales"),
+                                                   _dev(scale2, torch.float32, "scale2"),
+                                                   _dev(out, torch.bfloat16, "out"), E, N, K, _stream(stream))
+    _check("nvfp4_dequantize_from_host", rc)
     return out
 
 

@@ -12,11 +12,41 @@
 // banks: no conflicts); values are scaled by an exact fp32 power of two and
 // rounded to bf16, which never rounds for scale bytes <= 252 and gives the bf16
 // subnormals / infinities of the exact product for the extreme bytes.
+//
+// Both decode kernels also serve dequant-on-copy from host memory (kHostSrc): the
+// packed bank stays in page-locked host memory, the kernel reads it through its
+// device mapping with plain coherent loads, so only the packed codes cross the host
+// link and the bf16 weights land directly in device memory.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
+// Packed-bank reads: the read-only path for device memory, plain global loads for
+// mapped host memory.
+template <bool kHostSrc>
+__device__ __forceinline__ uint32_t load_word(const uint32_t *p) {
+    if constexpr (kHostSrc) {
+        uint32_t v;
+        asm volatile("ld.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+        return v;
+    } else {
+        return __ldg(p);
+    }
+}
+
+template <bool kHostSrc>
+__device__ __forceinline__ uint32_t load_byte(const uint8_t *p) {
+    if constexpr (kHostSrc) {
+        uint32_t v;
+        asm volatile("ld.global.u8 %0, [%1];" : "=r"(v) : "l"(p));
+        return v;
+    } else {
+        return __ldg(p);
+    }
+}
+
+template <bool kHostSrc>
 __global__ void __launch_bounds__(256) mxfp4_dequant_kernel(const uint32_t *__restrict__ packed,
                                                             const uint8_t *__restrict__ scales,
                                                             uint4 *__restrict__ out,
@@ -37,8 +67,8 @@ __global__ void __launch_bounds__(256) mxfp4_dequant_kernel(const uint32_t *__re
         uint32_t word[U], s[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            word[u] = __ldg(packed + w + u * stride);
-            s[u] = __ldg(scales + ((w + u * stride) >> 2));  // 4 words per 32-element block
+            word[u] = load_word<kHostSrc>(packed + w + u * stride);
+            s[u] = load_byte<kHostSrc>(scales + ((w + u * stride) >> 2));  // 4 words per 32-element block
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -58,8 +88,8 @@ __global__ void __launch_bounds__(256) mxfp4_dequant_kernel(const uint32_t *__re
         }
     }
     for (; w < n_words; w += stride) {
-        const uint32_t q = __ldg(packed + w);
-        const uint32_t sb = __ldg(scales + (w >> 2));
+        const uint32_t q = load_word<kHostSrc>(packed + w);
+        const uint32_t sb = load_byte<kHostSrc>(scales + (w >> 2));
         uint4 v;
         if (sb == 255u) {
             raise_device_error(MOE_DEVERR_BAD_SCALE);
@@ -155,6 +185,7 @@ __device__ __forceinline__ uint4 nvfp4_word(uint32_t q, uint32_t sb, const float
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+template <bool kHostSrc>
 __global__ void __launch_bounds__(256) nvfp4_dequant_kernel(const uint32_t *__restrict__ packed,
                                                             const uint8_t *__restrict__ scales,
                                                             const float *__restrict__ scale2,
@@ -180,14 +211,15 @@ __global__ void __launch_bounds__(256) nvfp4_dequant_kernel(const uint32_t *__re
             uint32_t word[U], sb[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                word[u] = __ldg(src + w + u * stride);
-                sb[u] = __ldg(sc_e + ((w + u * stride) >> 1));
+                word[u] = load_word<kHostSrc>(src + w + u * stride);
+                sb[u] = load_byte<kHostSrc>(sc_e + ((w + u * stride) >> 1));
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) __stcs(dst + w + u * stride, nvfp4_word(word[u], sb[u], lut, s2, mode));
         }
         for (; w < words_per_expert; w += stride)
-            __stcs(dst + w, nvfp4_word(__ldg(src + w), __ldg(sc_e + (w >> 1)), lut, s2, mode));
+            __stcs(dst + w, nvfp4_word(load_word<kHostSrc>(src + w), load_byte<kHostSrc>(sc_e + (w >> 1)), lut,
+                                       s2, mode));
     }
 }
 

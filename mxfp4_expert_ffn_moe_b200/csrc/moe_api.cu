@@ -497,6 +497,77 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     return rc;
 }
 
+// Standalone decode of a packed bank to bf16; kHostSrc: blocks and scales are the
+// device mappings of page-locked host memory.
+template <bool kHostSrc>
+int launch_mxfp4_dequant(const uint8_t *blocks, const uint8_t *scales, uint16_t *out, int64_t E, int64_t N,
+                         int64_t K, cudaStream_t stream) {
+    if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || N < 1 || K < 32 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(blocks, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    const int64_t n_words = E * N * (K / 8);
+    const int threads = 256;
+    int64_t blocks_needed = (n_words + threads - 1) / threads;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
+    StageScope scope(MOE_STAGE_DEQUANT, stream);
+    moe::mxfp4_dequant_kernel<kHostSrc><<<grid, threads, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(blocks), scales, reinterpret_cast<uint4 *>(out), n_words);
+    return launch_check();
+}
+
+template <bool kHostSrc>
+int launch_nvfp4_dequant(const uint8_t *blocks, const uint8_t *scales, const float *scale2, uint16_t *out,
+                         int64_t E, int64_t N, int64_t K, cudaStream_t stream) {
+    if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
+    if (E < 1 || N < 1 || K < 16 || K % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(blocks, 16) || !aligned(out, 16) || !aligned(scale2, 4)) return MOE_ERR_INVALID_ARG;
+    const int64_t words_per_expert = N * (K / 8);
+    const int threads = 256;
+    // one wave: as many blocks as the SMs hold at once, spread over the experts
+    static int per_sm = 0;
+    if (per_sm == 0 &&
+        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::nvfp4_dequant_kernel<kHostSrc>, threads, 0) !=
+             cudaSuccess || per_sm < 1))
+        per_sm = 4;
+    const int64_t target = (int64_t)sm_count() * per_sm;
+    const int64_t gy = E < 65535 ? E : 65535;
+    int64_t gx = target / gy;
+    const int64_t need_x = moe::ceil_div(words_per_expert, threads);
+    if (gx > need_x) gx = need_x;
+    if (gx < 1) gx = 1;
+    StageScope scope(MOE_STAGE_DEQUANT, stream);
+    moe::nvfp4_dequant_kernel<kHostSrc><<<dim3((unsigned)gx, (unsigned)gy), threads, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(blocks), scales, scale2, reinterpret_cast<uint4 *>(out),
+        words_per_expert, E);
+    return launch_check();
+}
+
+// Dequant-on-copy from host memory (MoE-Infinity PR #152: fetched packed experts are
+// dequantised on copy): the device address of `bytes` of page-locked host memory, or
+// an error when the first or the last byte is not host memory the current device can
+// address, or the two are not mapped contiguously.
+int device_view_of_host(const void *host, int64_t bytes, const void **dev) {
+    if (!host || bytes < 1) return MOE_ERR_INVALID_ARG;
+    const char *first = static_cast<const char *>(host);
+    const char *last = first + (bytes - 1);
+    cudaPointerAttributes a, b;
+    if (cudaPointerGetAttributes(&a, first) != cudaSuccess || cudaPointerGetAttributes(&b, last) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_INVALID_ARG;
+    }
+    if (a.type != cudaMemoryTypeHost || b.type != cudaMemoryTypeHost || !a.devicePointer || !b.devicePointer)
+        return MOE_ERR_INVALID_ARG;
+    if (static_cast<const char *>(b.devicePointer) != static_cast<const char *>(a.devicePointer) + (bytes - 1))
+        return MOE_ERR_INVALID_ARG;
+    *dev = a.devicePointer;
+    return MOE_OK;
+}
+
+bool bank_sizes_ok(int64_t E, int64_t N, int64_t K, int64_t block) {
+    return E >= 1 && N >= 1 && K >= block && K % block == 0 && E <= (int64_t(1) << 40) / N / K;
+}
+
 }  // namespace
 
 extern "C" {
@@ -515,44 +586,35 @@ const char *moe_status_string(int status) {
 
 int mxfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out, int64_t E,
                      int64_t N, int64_t K, void *stream) {
-    if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
-    if (E < 1 || N < 1 || K < 32 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
-    if (!aligned(blocks, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
-    const int64_t n_words = E * N * (K / 8);
-    const int threads = 256;
-    int64_t blocks_needed = (n_words + threads - 1) / threads;
-    const int64_t cap = (int64_t)sm_count() * 8;
-    const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
-    StageScope scope(MOE_STAGE_DEQUANT, (cudaStream_t)stream);
-    moe::mxfp4_dequant_kernel<<<grid, threads, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<const uint32_t *>(blocks), scales, reinterpret_cast<uint4 *>(out), n_words);
-    return launch_check();
+    return launch_mxfp4_dequant<false>(blocks, scales, out, E, N, K, (cudaStream_t)stream);
 }
 
 int nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2, uint16_t *out,
                      int64_t E, int64_t N, int64_t K, void *stream) {
-    if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
-    if (E < 1 || N < 1 || K < 16 || K % 16 != 0) return MOE_ERR_INVALID_ARG;
-    if (!aligned(blocks, 16) || !aligned(out, 16) || !aligned(scale2, 4)) return MOE_ERR_INVALID_ARG;
-    const int64_t words_per_expert = N * (K / 8);
-    const int threads = 256;
-    // one wave: as many blocks as the SMs hold at once, spread over the experts
-    static int per_sm = 0;
-    if (per_sm == 0 &&
-        (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::nvfp4_dequant_kernel, threads, 0) !=
-             cudaSuccess || per_sm < 1))
-        per_sm = 4;
-    const int64_t target = (int64_t)sm_count() * per_sm;
-    const int64_t gy = E < 65535 ? E : 65535;
-    int64_t gx = target / gy;
-    const int64_t need_x = moe::ceil_div(words_per_expert, threads);
-    if (gx > need_x) gx = need_x;
-    if (gx < 1) gx = 1;
-    StageScope scope(MOE_STAGE_DEQUANT, (cudaStream_t)stream);
-    moe::nvfp4_dequant_kernel<<<dim3((unsigned)gx, (unsigned)gy), threads, 0, (cudaStream_t)stream>>>(
-        reinterpret_cast<const uint32_t *>(blocks), scales, scale2, reinterpret_cast<uint4 *>(out),
-        words_per_expert, E);
-    return launch_check();
+    return launch_nvfp4_dequant<false>(blocks, scales, scale2, out, E, N, K, (cudaStream_t)stream);
+}
+
+int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales, uint16_t *out,
+                               int64_t E, int64_t N, int64_t K, void *stream) {
+    if (!bank_sizes_ok(E, N, K, 32)) return MOE_ERR_INVALID_ARG;
+    const void *db = nullptr, *ds = nullptr;
+    int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
+    if (rc == MOE_OK) rc = device_view_of_host(host_scales, E * N * (K / 32), &ds);
+    if (rc != MOE_OK) return rc;
+    return launch_mxfp4_dequant<true>(static_cast<const uint8_t *>(db), static_cast<const uint8_t *>(ds), out, E,
+                                      N, K, (cudaStream_t)stream);
+}
+
+int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales,
+                               const float *scale2, uint16_t *out, int64_t E, int64_t N, int64_t K,
+                               void *stream) {
+    if (!bank_sizes_ok(E, N, K, 16)) return MOE_ERR_INVALID_ARG;
+    const void *db = nullptr, *ds = nullptr;
+    int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
+    if (rc == MOE_OK) rc = device_view_of_host(host_scales, E * N * (K / 16), &ds);
+    if (rc != MOE_OK) return rc;
+    return launch_nvfp4_dequant<true>(static_cast<const uint8_t *>(db), static_cast<const uint8_t *>(ds), scale2,
+                                      out, E, N, K, (cudaStream_t)stream);
 }
 
 int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *ids,
