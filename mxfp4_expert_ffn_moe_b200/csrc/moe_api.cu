@@ -596,7 +596,7 @@ int nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *
 
 int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales, uint16_t *out,
                                int64_t E, int64_t N, int64_t K, void *stream) {
-    if (!bank_sizes_ok(E, N, K, 32)) return MOE_ERR_INVALID_ARG;
+    if (!host_blocks || !host_scales || !out || !bank_sizes_ok(E, N, K, 32)) return MOE_ERR_INVALID_ARG;
     const void *db = nullptr, *ds = nullptr;
     int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
     if (rc == MOE_OK) rc = device_view_of_host(host_scales, E * N * (K / 32), &ds);
@@ -608,7 +608,7 @@ int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_s
 int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales,
                                const float *scale2, uint16_t *out, int64_t E, int64_t N, int64_t K,
                                void *stream) {
-    if (!bank_sizes_ok(E, N, K, 16)) return MOE_ERR_INVALID_ARG;
+    if (!host_blocks || !host_scales || !out || !bank_sizes_ok(E, N, K, 16)) return MOE_ERR_INVALID_ARG;
     const void *db = nullptr, *ds = nullptr;
     int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
     if (rc == MOE_OK) rc = device_view_of_host(host_scales, E * N * (K / 16), &ds);

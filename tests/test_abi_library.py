@@ -99,3 +99,43 @@ def test_profiler_stage_mask_host_logic(lib):
     assert lib.moe_profile_read(ms, launches) == 0
     with pytest.raises(ValueError):
         moe.moe_profile_enable_stages(["no_such_stage"])
+
+
+def test_nvfp4_router_and_host_copy_argument_checks_need_no_device(lib):
+    # The NVFP4, router and host-copy entry points reject bad calls in the host-side
+    # validation, before any CUDA call.
+    p = ctypes.c_void_p(0x1000)          # never dereferenced
+    null = None
+    # nvfp4_dequantize
+    assert lib.nvfp4_dequantize(null, p, null, p, 1, 1, 16, null) == -1
+    assert lib.nvfp4_dequantize(p, p, null, p, 1, 1, 24, null) == -1                    # K % 16
+    assert lib.nvfp4_dequantize(p, p, ctypes.c_void_p(0x1002), p, 1, 1, 16, null) == -1  # scale2 alignment
+    # moe_nvfp4_forward_ex: x, T, H, I, E, k, ids, w, gu blocks/scales/scale2/bias, d blocks/scales/scale2/bias
+    args = [p, 8, 128, 128, 4, 2, p, p, p, p, None, None, p, p, None, None, ctypes.c_float(1.702),
+            ctypes.c_float(7.0), p, ctypes.c_uint32(0), None, 0, null]
+    bad = list(args)
+    bad[0] = None
+    assert lib.moe_nvfp4_forward_ex(*bad) == -1
+    bad = list(args)
+    bad[2] = 96                                                                             # H % 64
+    assert lib.moe_nvfp4_forward_ex(*bad) == -1
+    bad = list(args)
+    bad[11], bad[19] = p, ctypes.c_uint32(1)                         # weight on input with a bias
+    assert lib.moe_nvfp4_forward_ex(*bad) == -1
+    bad = list(args)
+    bad[10] = ctypes.c_void_p(0x1002)                                                       # scale2 alignment
+    assert lib.moe_nvfp4_forward_ex(*bad) == -1
+    bad = list(args)
+    bad[20], bad[21] = ctypes.c_void_p(0x100000), 64                                        # workspace too small
+    assert lib.moe_nvfp4_forward_ex(*bad) == -4
+    # moe_router_route: x, w, b, T, H, E, k, logits, ids, weights
+    assert lib.moe_router_route(null, p, null, 8, 128, 32, 4, null, p, p, null) == -1
+    assert lib.moe_router_route(p, p, null, 8, 96, 32, 4, null, p, p, null) == -1          # H % 64
+    assert lib.moe_router_route(p, p, null, 8, 128, 4, 5, null, p, p, null) == -1          # k > E
+    assert lib.moe_router_route(p, p, null, 8, 128, 300, 4, null, p, p, null) == -2        # E > 256
+    assert lib.moe_router_route(ctypes.c_void_p(0x1008), p, null, 8, 128, 32, 4, null, p, p, null) == -1
+    # *_dequantize_from_host: sizes are checked before the host pointers are looked at
+    assert lib.mxfp4_dequantize_from_host(p, p, p, 1, 1, 48, null) == -1                  # K % 32
+    assert lib.mxfp4_dequantize_from_host(null, p, p, 1, 1, 32, null) == -1
+    assert lib.nvfp4_dequantize_from_host(p, p, null, p, 1, 1, 24, null) == -1            # K % 16
+    assert lib.nvfp4_dequantize_from_host(p, null, null, p, 1, 1, 16, null) == -1
