@@ -443,10 +443,18 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     int rc = MOE_OK;
     do {
         {
-            const size_t perm_smem = sizeof(int) * (32 * E + E + 1);
+            // stage the ids in shared memory when they fit (up to ~50K pairs)
+            static bool perm_attr = false;
+            if (!perm_attr) {
+                perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)moe::kPermuteSmemCap) == cudaSuccess;
+                if (!perm_attr) cudaGetLastError();
+            }
+            const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
+            const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
             StageScope sp(MOE_STAGE_PERMUTE, s);
             launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P,
-                       (int)E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs);
+                       (int)E, config_tok(cfg), staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs);
         }
         if ((rc = launch_check()) != MOE_OK) break;
         const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
@@ -659,15 +667,17 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
     cudaStream_t s = (cudaStream_t)stream;
     CUtensorMap mx, mw;
     if (!make_act_map(&mx, x, T, H) || !make_act_map(&mw, w_router, E, H)) return MOE_ERR_CUDA;
-    const uint32_t smem = moe::rtr::smem_bytes((int)E);
+    const int slots = moe::rtr::ring_slots((int)E);
+    const uint32_t smem = moe::rtr::smem_bytes((int)E, slots);
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(moe::rtr::router_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    auto kernel = slots == 8 ? moe::rtr::router_route_kernel<8>
+                  : slots == 6 ? moe::rtr::router_route_kernel<6> : moe::rtr::router_route_kernel<4>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     const int64_t grid = moe::ceil_div(T, moe::rtr::BM);
     StageScope scope(MOE_STAGE_ROUTE, s);
-    launch_pdl(moe::rtr::router_route_kernel, dim3((unsigned)grid), dim3(moe::rtr::kThreads), smem, s, mx, mw,
-               b_router, (int)T, (int)H, (int)E, k, logits, ids, weights);
+    launch_pdl(kernel, dim3((unsigned)grid), dim3(moe::rtr::kThreads), smem, s, mx, mw, b_router, (int)T, (int)H,
+               (int)E, k, logits, ids, weights);
     return launch_check();
 }
 

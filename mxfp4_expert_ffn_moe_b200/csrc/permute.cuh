@@ -13,7 +13,9 @@
 // One CTA of 32 warps: warp w owns a contiguous chunk of pairs, counts its experts
 // in a private shared-memory row, the chunk bases come from an exclusive scan over
 // warps, and each warp then scatters its chunk in order using __match_any_sync to
-// rank equal experts inside a 32-pair step.
+// rank equal experts inside a 32-pair step.  When the ids fit (staged != 0) they are
+// first copied into shared memory with independent, coalesced loads, so neither
+// pass over them waits on a global load per step.
 #pragma once
 #include "common.cuh"
 
@@ -21,8 +23,15 @@ namespace moe {
 
 constexpr int kPermuteThreads = 1024;
 
+// Dynamic shared memory of permute_pairs_kernel: the count rows and expert starts,
+// plus P staged ids when `staged`.
+__host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t P, bool staged) {
+    return sizeof(int) * (size_t)(32 * E + E + 1) + (staged ? sizeof(int) * (size_t)P : 0);
+}
+constexpr size_t kPermuteSmemCap = 200 * 1024;
+
 __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
-    const int32_t *__restrict__ ids, int64_t P, int E, int bm, int32_t *__restrict__ counts,
+    const int32_t *__restrict__ ids, int64_t P, int E, int bm, int staged, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
     int32_t *__restrict__ sorted_pairs) {
     pdl_wait();
@@ -30,15 +39,19 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     extern __shared__ int sm_perm[];
     int *cnt = sm_perm;             // [32][E]: per-warp counts, then per-warp running bases
     int *off = sm_perm + 32 * E;    // [E + 1]: expert start rows
+    int *ids_s = off + E + 1;       // [P] when staged
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
+    if (staged)
+        for (int64_t i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = __ldg(ids + i);
     __syncthreads();
+    const int32_t *src = staged ? ids_s : ids;
 
     const int64_t chunk = (P + 31) / 32;
     const int64_t beg = (int64_t)warp * chunk;
     const int64_t end = (beg + chunk < P) ? beg + chunk : P;
     for (int64_t p = beg + lane; p < end; p += 32) {
-        const int e = ids[p];
+        const int e = src[p];
         if ((unsigned)e < (unsigned)E)
             atomicAdd(&cnt[warp * E + e], 1);
         else
@@ -73,7 +86,7 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     __syncthreads();
     for (int64_t base = beg; base < end; base += 32) {
         const int64_t p = base + lane;
-        const int e = (p < end) ? ids[p] : -1;
+        const int e = (p < end) ? src[p] : -1;
         const bool valid = (p < end) && (unsigned)e < (unsigned)E;
         const int key = valid ? e : -1 - lane;
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);

@@ -11,7 +11,9 @@
 // router rows (padded to a multiple of 32, at most 256) on N, so the whole logit row
 // of a token ends up in one thread's TMEM lane:
 //   warp 0     TMA: per K step of 64, the token tile (32-row boxes, 128-byte swizzle)
-//              and the router rows (same boxes), into an S-slot ring
+//              and the router rows (same boxes), into an S-slot ring (S = 8, 6, 4 for
+//              E up to 64, 128, 256: about 192 KB, enough loads in flight to cover
+//              the HBM round trip of the small per-step boxes)
 //   warp 1     TMEM owner and MMA issuer: 4 x tcgen05.mma 128 x E_pad x 16 per step
 //   warps 2-5  epilogue, one token per thread (TMEM lane quarter = warp % 4): reads
 //              its logits 32 columns at a time, adds the bias, optionally stores the
@@ -28,7 +30,6 @@ namespace rtr {
 
 constexpr int BM = 128;                          // tokens per tile (TMEM lanes)
 constexpr int BK = 64;                           // K elements per step (128-byte rows)
-constexpr int S = 4;                             // ring slots
 constexpr int kThreads = 192;
 constexpr uint32_t BOX_ROWS = 32;
 constexpr uint32_t BOX_BYTES = BOX_ROWS * BK * 2;   // 4096
@@ -40,9 +41,11 @@ __host__ __device__ constexpr uint32_t stage_bytes(int E) { return A_BYTES + (ui
 __host__ __device__ constexpr uint32_t tmem_cols(int E) {
     return e_pad(E) <= 32 ? 32u : e_pad(E) <= 64 ? 64u : e_pad(E) <= 128 ? 128u : 256u;
 }
+__host__ __device__ constexpr int ring_slots(int E) { return e_pad(E) <= 64 ? 8 : e_pad(E) <= 128 ? 6 : 4; }
 // ring + barriers (2 S + 1) + TMEM holder + 1 KB alignment slack
-__host__ __device__ constexpr uint32_t smem_bytes(int E) { return S * stage_bytes(E) + 8 * (2 * S + 2) + 1024; }
+__host__ __device__ constexpr uint32_t smem_bytes(int E, int S) { return S * stage_bytes(E) + 8 * (2 * S + 2) + 1024; }
 
+template <int S>
 __global__ void __launch_bounds__(kThreads, 1)
     router_route_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                         const float *__restrict__ bias, int T, int H, int E, int k,
