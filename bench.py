@@ -219,6 +219,24 @@ def time_steps(fn, steps, stream, flush=None):
     return total
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its device time and all get the
+    max (NCCL on the GPUs; any backend whose tensors live on `device`)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time (weak scaling:
+    each replica runs the full workload)."""
+    return world * tokens_per_rank * steps / (ms_max * 1e-3)
+
+
 def graph_of(fn, stream):
     """fn captured into a CUDA graph (the library's launches, programmatic dependent
     launch edges included), or None with the reason when capture is not possible."""
@@ -562,11 +580,8 @@ def run_ours(args):
     ms_total = ev0.elapsed_time(ev1)
     ms_profiled = ev2.elapsed_time(ev3)
     prof = moe.moe_profile_read()
-    if world > 1:
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
-    value = world * L.T * args.steps / (ms_total * 1e-3)
+    ms_total = max_over_ranks(ms_total, world, device)
+    value = job_throughput(L.T, args.steps, world, ms_total)
     gpu_launches = sum(v[1] for v in launches.values())
 
     # end to end through the public API: pinned host inputs -> device -> layer -> host.
@@ -618,11 +633,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     moe.moe_profile_read()
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * L.T * e2e_steps / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
+    e2e_value = job_throughput(L.T, e2e_steps, world, e2e_ms)
 
     # roofline of the dominant kernel (gate_up grouped GEMM), from the live events
     gu_ms, gu_n = prof["gate_up"]

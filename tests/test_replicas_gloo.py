@@ -1,0 +1,70 @@
+"""The N > 1 path of the benchmark on CPU: two gloo ranks (world size 2) run the
+replica bookkeeping that bench.py does over NCCL on GPUs -- max over ranks of the
+device time, whole-job throughput, rank-0-only output -- and the reference arm's
+non-zero ranks exit without work.  No GPU."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    sys.path.insert(0, ROOT)
+    import bench
+    ms = 10.0 + 5.0 * rank                       # rank 1 is the slower replica
+    got = bench.max_over_ranks(ms, world, "cpu")
+    value = bench.job_throughput(4096, 20, world, got)
+    dist.barrier()
+    q.put((rank, got, value))
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_max_over_ranks_and_throughput_two_gloo_ranks():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(150)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, got, value in res:
+        assert got == 15.0                        # every rank sees the slowest time
+        assert value == pytest.approx(2 * 4096 * 20 / 15e-3)
+
+
+def test_single_rank_is_the_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(12.5, 1, "cpu") == 12.5
+    assert bench.job_throughput(4096, 10, 1, 10.0) == pytest.approx(4096 * 10 / 10e-3)
+
+
+@pytest.mark.timeout(120)
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], env=env, capture_output=True, text=True, timeout=100)
+    assert r.returncode == 0, r.stderr[-500:]
+    assert r.stdout.strip() == ""
