@@ -443,13 +443,12 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     int rc = MOE_OK;
     do {
         {
-            // stage the ids in shared memory when they fit (up to ~50K pairs)
-            static bool perm_attr = false;
-            if (!perm_attr) {
-                perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)moe::kPermuteSmemCap) == cudaSuccess;
-                if (!perm_attr) cudaGetLastError();
-            }
+            // stage the ids in shared memory when they fit (up to ~50K pairs); the
+            // attribute is per device, so it is set on every call, like the GEMMs'
+            const bool perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        (int)moe::kPermuteSmemCap) == cudaSuccess;
+            if (!perm_attr) cudaGetLastError();
             const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
             const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
             StageScope sp(MOE_STAGE_PERMUTE, s);
