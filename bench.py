@@ -21,6 +21,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -76,7 +77,8 @@ class ClockSampler:
     def __init__(self, device_id: str):
         self.device_id = device_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        # raw samples go to a temporary file; the summary rides in the JSON line
+        self.path = os.path.join(tempfile.gettempdir(), f"moe_bench_clocks_{os.getpid()}.csv")
         self.window = None
 
     def mark(self, t0: float, t1: float):

@@ -59,7 +59,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = -1, /* null pointer, bad size, misalignment, bad flag mix */
-    MOE_ERR_UNSUPPORTED = -2, /* valid but outside what this build implements      */
+    MOE_ERR_UNSUPPORTED = -2, /* valid but outside what the library implements     */
     MOE_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed               */
     MOE_ERR_NO_MEMORY = -4,   /* workspace allocation failed or workspace too small */
     MOE_ERR_DEVICE = -5       /* the sticky device error word is set                */
