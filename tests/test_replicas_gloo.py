@@ -68,3 +68,27 @@ def test_reference_arm_other_ranks_exit_without_work():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=100)
     assert r.returncode == 0, r.stderr[-500:]
     assert r.stdout.strip() == ""
+
+
+@pytest.mark.timeout(120)
+def test_reference_arm_json_line_contract():
+    # the reference arm (the CPU oracle on the host cores) prints one JSON line with the
+    # contract's keys; run on the tiny layer so that it takes a second
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "2",
+                        "--warmup", "3", "--workload", "tiny_woo"], env=env, capture_output=True, text=True,
+                       timeout=100)
+    assert r.returncode == 0, r.stderr[-500:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["config"]["workload"] == "tiny_woo"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
