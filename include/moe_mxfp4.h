@@ -70,6 +70,9 @@ typedef enum {
 #define MOE_DEVERR_BAD_SCALE 0x2     /* an E8M0 byte 0xff, or an E4M3 NaN byte
                                         (0x7f / 0xff), was decoded                  */
 #define MOE_DEVERR_TIMEOUT 0x4       /* a bounded pipeline wait gave up              */
+#define MOE_DEVERR_BAD_LOGIT 0x8     /* a token had fewer than k non-NaN router logits */
+#define MOE_DEVERR_OUT_OF_BOUNDS 0x10 /* bounds-checked builds only: an index fell
+                                        outside its buffer (the access was skipped) */
 
 /* moe_mxfp4_forward_ex flags */
 #define MOE_FLAG_WEIGHT_ON_INPUT 0x1u /* router weight scales each expert's input  */
@@ -117,7 +120,11 @@ int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_s
  *                    expert index;
  *   weights[t, j]    exp(l_j - l_max) / sum over the k chosen of exp(l_i - l_max).
  *   router_logits fp32 [T, E]; ids int32 [T, k]; weights fp32 [T, k].
- * Sizes: T >= 1, 1 <= E <= 256, 1 <= k <= min(E, 8).  NaN logits are unsupported.
+ * Sizes: T >= 1, 1 <= E <= 256, 1 <= k <= min(E, 8).  NaN logits are never chosen:
+ * a token with fewer than k non-NaN logits gets id -1 and weight 0 in its remaining
+ * slots (the softmax runs over the chosen logits only) and MOE_DEVERR_BAD_LOGIT is
+ * raised; the forward calls then drop those slots (and raise
+ * MOE_DEVERR_BAD_EXPERT_ID).
  */
 int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *ids,
               float *weights, void *stream);
@@ -186,6 +193,35 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
 /* Bytes of workspace moe_mxfp4_forward_ex (and moe_nvfp4_forward_ex) needs for
  * these sizes (0 on bad sizes). */
 size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int k);
+
+/*
+ * moe_token_tile_rows -- the token-tile height (rows of one expert per tile of the
+ * grouped GEMMs) that moe_mxfp4_forward_ex (nvfp4 = 0) or moe_nvfp4_forward_ex
+ * (nvfp4 != 0) uses for these sizes on the current device, or MOE_ERR_INVALID_ARG
+ * for sizes the forward refuses.  Host-only; enqueues nothing.
+ */
+int moe_token_tile_rows(int64_t T, int64_t H, int64_t I, int64_t E, int k, int nvfp4);
+
+/*
+ * moe_permute -- the layer's grouping of (token, slot) pairs by expert, on its own
+ * (FreeToken PR #838, "What it does": expert-ordered prefill views; the gather of
+ * [T, k, 2I] rows its review names).  Pair p = t*k + j is routed to ids[p]:
+ *   ids           int32 [T, k]
+ *   counts        int32 [E]      pairs per expert
+ *   offsets       int32 [E + 1]  exclusive scan of counts; offsets[E] = valid pairs
+ *   tile_offsets  int32 [E + 1]  the same scan over ceil(counts[e] / tile_rows)
+ *   sorted_pairs  int32 [T*k]    row r (expert order) holds its pair p; inside one
+ *                                expert the rows follow ascending p (stable); rows
+ *                                past offsets[E] are left untouched
+ *   pair_rows     int32 [T*k] or NULL: the inverse, the row of pair p (-1 when the
+ *                                pair was dropped)
+ * Ids outside [0, E) drop their pair and raise MOE_DEVERR_BAD_EXPERT_ID.  Sizes:
+ * T >= 1; 1 <= k <= 8; 1 <= E <= 256; tile_rows >= 1; T*k < 2^31.  Errors:
+ * MOE_ERR_INVALID_ARG for null pointers or sizes.
+ */
+int moe_permute(const int32_t *ids, int64_t T, int k, int64_t E, int tile_rows, int32_t *counts,
+                int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
+                void *stream);
 
 /*
  * NVFP4 expert banks: the packed E2M1 codes of the MXFP4 layout with one E4M3 scale
@@ -261,7 +297,10 @@ int moe_get_device_error(void *stream);
  *   is enqueued (for H = I = 2880 and k = 4 that is about 340 tokens).
  *   The first call on a device looks up the array's device address on that
  *   device (cudaGetSymbolAddress, with the device current); make that first call
- *   before any stream capture.  Later calls on the device reuse the address.
+ *   before any stream capture.  Later calls on the device reuse the address while
+ *   the device's context stays the same; after the context is destroyed and made
+ *   again (cudaDeviceReset) the next call looks it up anew, so make that call
+ *   outside stream capture too.
  *   Every call on a device shares the one array, which keeps the previous call's
  *   contents; the layer writes every scratch byte before it reads it, so nothing
  *   needs clearing.  Calls whose work overlaps on the GPU (different streams

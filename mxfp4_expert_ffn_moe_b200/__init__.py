@@ -22,7 +22,8 @@ __all__ = [
     "moe_profile_read",
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
-    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host",
+    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host", "moe_permute", "moe_token_tile_rows",
+    "MOE_DEVERR_BAD_LOGIT", "MOE_DEVERR_OUT_OF_BOUNDS",
 ]
 
 MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -31,13 +32,15 @@ MOE_FLAG_WEIGHT_ON_INPUT = 0x1
 MOE_DEVERR_BAD_EXPERT_ID = 0x1
 MOE_DEVERR_BAD_SCALE = 0x2
 MOE_DEVERR_TIMEOUT = 0x4
+MOE_DEVERR_BAD_LOGIT = 0x8
+MOE_DEVERR_OUT_OF_BOUNDS = 0x10
 
 EXPORTED_SYMBOLS = (
     "mxfp4_dequantize", "moe_route", "moe_mxfp4_forward", "moe_mxfp4_forward_ex",
     "moe_mxfp4_workspace_size", "moe_status_string", "moe_get_device_error",
     "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
-    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host",
+    "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host", "moe_permute", "moe_token_tile_rows",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
@@ -98,6 +101,10 @@ def load_library():
               ctypes.c_float, p, ctypes.c_uint32, p, ctypes.c_size_t, p]
     lib.moe_nvfp4_forward_ex.argtypes = nv_fwd
     lib.moe_nvfp4_forward_ex.restype = i32
+    lib.moe_permute.argtypes = [p, i64, i32, i64, i32, p, p, p, p, p, p]
+    lib.moe_permute.restype = i32
+    lib.moe_token_tile_rows.argtypes = [i64, i64, i64, i64, i32, i32]
+    lib.moe_token_tile_rows.restype = i32
     lib.moe_profile_read.argtypes = [p, p]
     lib.moe_profile_read.restype = i32
     _lib = lib
@@ -314,6 +321,34 @@ def moe_nvfp4_forward_ex(x, ids, weights, gate_up_blocks, gate_up_scales, gate_u
         _dev(out, torch.bfloat16, "out"), ctypes.c_uint32(flags), ws, nbytes, _stream(stream))
     _check("moe_nvfp4_forward_ex", rc)
     return out
+
+
+def moe_permute(ids, E: int, tile_rows: int, want_pair_rows: bool = True, stream=None):
+    """Group the (token, slot) pairs of int32 ids [T, k] by expert.  Returns a dict of
+    int32 device tensors: counts [E], offsets [E + 1], tile_offsets [E + 1],
+    sorted_pairs [T*k] and (with want_pair_rows) pair_rows [T*k]."""
+    import torch
+    T, k = ids.shape
+    dev = ids.device
+    out = {"counts": torch.empty(E, dtype=torch.int32, device=dev),
+           "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+           "tile_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+           "sorted_pairs": torch.empty(T * k, dtype=torch.int32, device=dev)}
+    if want_pair_rows:
+        out["pair_rows"] = torch.empty(T * k, dtype=torch.int32, device=dev)
+    rc = load_library().moe_permute(
+        _dev(ids, torch.int32, "ids"), T, int(k), int(E), int(tile_rows),
+        *[_dev(out[n], torch.int32, n) for n in ("counts", "offsets", "tile_offsets", "sorted_pairs")],
+        _dev(out.get("pair_rows"), torch.int32, "pair_rows"), _stream(stream))
+    _check("moe_permute", rc)
+    return out
+
+
+def moe_token_tile_rows(T: int, H: int, I: int, E: int, k: int, nvfp4: bool = False) -> int:
+    """Token-tile height the forward uses for these sizes on the current device."""
+    rc = int(load_library().moe_token_tile_rows(T, H, I, E, k, 1 if nvfp4 else 0))
+    _check("moe_token_tile_rows", rc if rc < 0 else 0)
+    return rc
 
 
 def moe_mxfp4_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:

@@ -8,6 +8,8 @@
 #define MOE_DEVERR_BAD_EXPERT_ID 0x1
 #define MOE_DEVERR_BAD_SCALE 0x2
 #define MOE_DEVERR_TIMEOUT 0x4
+#define MOE_DEVERR_BAD_LOGIT 0x8
+#define MOE_DEVERR_OUT_OF_BOUNDS 0x10
 
 namespace moe {
 

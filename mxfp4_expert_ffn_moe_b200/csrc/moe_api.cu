@@ -394,6 +394,22 @@ int config_tok(TileConfig c) {
     }
 }
 
+// Pair permutation (one CTA).  The ids are staged in shared memory when they fit (up
+// to ~50K pairs); the attribute is per device, so it is set on every call, like the
+// GEMMs'.
+int launch_permute(const int32_t *ids, int64_t P, int64_t E, int tile_rows, int32_t *counts, int32_t *offsets,
+                   int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows, cudaStream_t s) {
+    const bool perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)moe::kPermuteSmemCap) == cudaSuccess;
+    if (!perm_attr) cudaGetLastError();
+    const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
+    const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
+    StageScope sp(MOE_STAGE_PERMUTE, s);
+    launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P, (int)E,
+               tile_rows, staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs, pair_rows);
+    return launch_check();
+}
+
 // The whole layer on the caller's stream: permute -> gather (or split) -> gate_up ->
 // down -> combine.  nv: NVFP4 banks (E4M3 scales per 16 elements, weight_scale_2).
 int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
@@ -442,20 +458,9 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     const TileConfig cfg = pick_config(P, H, I, E, nv);
     int rc = MOE_OK;
     do {
-        {
-            // stage the ids in shared memory when they fit (up to ~50K pairs); the
-            // attribute is per device, so it is set on every call, like the GEMMs'
-            const bool perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                        (int)moe::kPermuteSmemCap) == cudaSuccess;
-            if (!perm_attr) cudaGetLastError();
-            const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
-            const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
-            StageScope sp(MOE_STAGE_PERMUTE, s);
-            launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P,
-                       (int)E, config_tok(cfg), staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs);
-        }
-        if ((rc = launch_check()) != MOE_OK) break;
+        if ((rc = launch_permute(ids, P, E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs,
+                                 nullptr, s)) != MOE_OK)
+            break;
         const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
         if (mxf) {
             uint8_t *xq = reinterpret_cast<uint8_t *>(x_perm);
@@ -678,6 +683,21 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
     launch_pdl(kernel, dim3((unsigned)grid), dim3(moe::rtr::kThreads), smem, s, mx, mw, b_router, (int)T, (int)H,
                (int)E, k, logits, ids, weights);
     return launch_check();
+}
+
+int moe_permute(const int32_t *ids, int64_t T, int k, int64_t E, int tile_rows, int32_t *counts,
+                int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
+                void *stream) {
+    if (!ids || !counts || !offsets || !tile_offsets || !sorted_pairs) return MOE_ERR_INVALID_ARG;
+    if (T < 1 || k < 1 || k > 8 || E < 1 || E > 256 || tile_rows < 1) return MOE_ERR_INVALID_ARG;
+    if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+    return launch_permute(ids, T * k, E, tile_rows, counts, offsets, tile_offsets, sorted_pairs, pair_rows,
+                          (cudaStream_t)stream);
+}
+
+int moe_token_tile_rows(int64_t T, int64_t H, int64_t I, int64_t E, int k, int nvfp4) {
+    if (!forward_sizes_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
+    return config_tok(pick_config(T * k, H, I, E, nvfp4 != 0));
 }
 
 size_t moe_mxfp4_workspace_size(int64_t T, int64_t H, int64_t I, int64_t E, int k) {

@@ -8,6 +8,7 @@
 //   tile_offsets[e]  first M-tile of expert e for an M-tile of bm rows
 //   sorted_pairs[r]  the pair p placed at row r; within an expert rows follow
 //                    ascending p (a stable, deterministic order)
+//   pair_rows[p]     (optional) the inverse: the row of pair p, -1 for a dropped pair
 // Ids outside [0, E) raise MOE_DEVERR_BAD_EXPERT_ID and their pairs are dropped.
 //
 // One CTA of 32 warps: warp w owns a contiguous chunk of pairs, counts its experts
@@ -33,7 +34,7 @@ constexpr size_t kPermuteSmemCap = 200 * 1024;
 __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     const int32_t *__restrict__ ids, int64_t P, int E, int bm, int staged, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
-    int32_t *__restrict__ sorted_pairs) {
+    int32_t *__restrict__ sorted_pairs, int32_t *__restrict__ pair_rows) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ int sm_perm[];
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
             sorted_pairs[off[e] + wbase + rank] = (int32_t)p;
             if (rank == 0) cnt[warp * E + e] = wbase + __popc(peers);
         }
+        if (pair_rows && p < end) pair_rows[p] = valid ? off[e] + wbase + rank : -1;
         __syncwarp();
     }
 }

@@ -8,6 +8,8 @@
 //
 // One warp per token; each lane holds VPL logits (expert lane + 32 v) in
 // registers, k rounds of a warp-wide arg-max with the (value desc, index asc) rule.
+// NaN logits are never chosen; a token with fewer than k other logits gets id -1
+// and weight 0 in its remaining slots and raises MOE_DEVERR_BAD_LOGIT.
 #pragma once
 #include "common.cuh"
 
@@ -56,20 +58,26 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                 bi = oi;
             }
         }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        // bi == E-or-more only when every remaining logit is NaN (a NaN never wins a
+        // comparison): the slot stays empty
+        if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
         sel_v[j] = bv;
         sel_i[j] = bi;
     }
     if (lane == 0) {
+        // empty slots (fewer than k non-NaN logits) get id -1 and weight 0 and flag
+        // the device error word; the softmax runs over the chosen logits only
         const float m = sel_v[0];
         float ex[8], sum = 0.0f;
         for (int j = 0; j < k; ++j) {
-            ex[j] = expf(sel_v[j] - m);
+            ex[j] = sel_i[j] < E ? expf(sel_v[j] - m) : 0.0f;
             sum += ex[j];
         }
-        const float inv = 1.0f / sum;
+        const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
         for (int j = 0; j < k; ++j) {
-            ids[t * k + j] = sel_i[j];
+            const bool valid = sel_i[j] < E;
+            if (!valid) raise_device_error(MOE_DEVERR_BAD_LOGIT);
+            ids[t * k + j] = valid ? sel_i[j] : -1;
             weights[t * k + j] = ex[j] * inv;
         }
     }

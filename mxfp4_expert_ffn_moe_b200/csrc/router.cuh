@@ -169,19 +169,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (live) {
-                // softmax over the k chosen, as the standalone routing kernel computes it
+                // softmax over the k chosen, as the standalone routing kernel computes it;
+                // a NaN logit never enters the list, so with fewer than k others a slot
+                // stays empty: id -1, weight 0, MOE_DEVERR_BAD_LOGIT
                 const float m = topv[0];
                 float ex[kMaxK], sum = 0.0f;
 #pragma unroll
                 for (int j = 0; j < kMaxK; ++j) {
-                    ex[j] = j < k ? expf(topv[j] - m) : 0.0f;
-                    if (j < k) sum += ex[j];
+                    ex[j] = (j < k && topi[j] < E) ? expf(topv[j] - m) : 0.0f;
+                    sum += ex[j];
                 }
-                const float inv = 1.0f / sum;
+                const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
 #pragma unroll
                 for (int j = 0; j < kMaxK; ++j) {
                     if (j < k) {
-                        ids[(int64_t)t * k + j] = topi[j];
+                        const bool valid = topi[j] < E;
+                        if (!valid) raise_device_error(MOE_DEVERR_BAD_LOGIT);
+                        ids[(int64_t)t * k + j] = valid ? topi[j] : -1;
                         weights[(int64_t)t * k + j] = ex[j] * inv;
                     }
                 }

@@ -39,17 +39,30 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 // One potentially blocking test of the phase: the hardware may suspend the
 // thread for up to `kSuspendNs` waiting for the phase to complete, so waiting
 // warps sleep instead of taking issue slots from the working ones.
-constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per try
+#ifndef MOE_MBAR_SUSPEND_NS
+#define MOE_MBAR_SUSPEND_NS 1000000
+#endif
+constexpr uint32_t kSuspendNs = MOE_MBAR_SUSPEND_NS;   // 0: no hint (implementation-defined limit)
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendNs)
-        : "memory");
+    if constexpr (kSuspendNs == 0) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
+            : "memory");
+    }
     return ok != 0;
 }
 
@@ -66,20 +79,23 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait until the phase of parity `parity` has completed.  Bounded: after tries
-// adding up to about four seconds (far beyond any legitimate wait of this
-// pipeline) it raises MOE_DEVERR_TIMEOUT and returns false so that the caller
-// can wind down instead of keeping the GPU busy forever.  The cycle counter is a
-// second bound in case a try returns early without the phase having completed.
+// Wait until the phase of parity `parity` has completed.  Bounded: after about
+// four seconds of clock cycles (far beyond any legitimate wait of this pipeline)
+// it raises MOE_DEVERR_TIMEOUT and returns false so that the caller can wind down
+// instead of keeping the GPU busy forever.  The try count is a second bound in case
+// the cycle counter misbehaves.  MOE_MBAR_SPIN polls with the non-blocking test
+// instead of the potentially blocking try.
 constexpr long long kWaitLimitCycles = 8000000000ll;
+#ifndef MOE_MBAR_SPIN
+#define MOE_MBAR_SPIN 0
+#endif
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (mbar_test_wait(bar, parity)) return true;
-    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
 #pragma unroll 1
-    for (uint32_t i = 1; i < 4000u; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < (1u << 27); ++i) {
+        if (MOE_MBAR_SPIN ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (clock64() - t0 > kWaitLimitCycles) break;
     }
     raise_device_error(MOE_DEVERR_TIMEOUT);

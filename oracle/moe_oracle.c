@@ -223,13 +223,15 @@ static double weight_elem_fmt(int fmt, const uint8_t *blocks, const uint8_t *sca
 void oracle_nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2,
                              uint16_t *out, int64_t E, int64_t N, int64_t K, int defect)
 {
-    for (int64_t e = 0; e < E; ++e) {
-        double s2 = scale2 ? (double)scale2[e] : 1.0;
-        for (int64_t n = 0; n < N; ++n)
+    /* rows are independent; OpenMP only spreads them over the host's cores */
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t e = 0; e < E; ++e)
+        for (int64_t n = 0; n < N; ++n) {
+            double s2 = scale2 ? (double)scale2[e] : 1.0;
             for (int64_t kk = 0; kk < K; ++kk)
                 out[(e * N + n) * K + kk] = oracle_double_to_bf16(
                     weight_elem_nvfp4(blocks, scales, N, K, e, n, kk, defect) * s2);
-    }
+        }
 }
 
 /* ---- standalone dequant-on-copy [P2] Changes ------------------------------- */
@@ -238,6 +240,8 @@ void oracle_nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const
 void oracle_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out,
                        int64_t E, int64_t N, int64_t K, int defect)
 {
+    /* rows are independent; OpenMP only spreads them over the host's cores */
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t e = 0; e < E; ++e)
         for (int64_t n = 0; n < N; ++n)
             for (int64_t kk = 0; kk < K; ++kk)

@@ -94,3 +94,27 @@ def sample_tokens(T, n, seed=0):
     rng = np.random.default_rng(seed)
     mid = rng.choice(np.arange(1, T - 1), size=n - 2, replace=False)
     return np.sort(np.concatenate([[0, T - 1], mid])).astype(np.int64)
+
+
+def stratified_tokens(ids, E, tile_rows, extra=8, seed=0):
+    """Tokens to compare at full size, chosen so that the sample reaches every tile the
+    grouped kernels form: pairs p = t*k + j are grouped by expert in ascending p (the
+    permutation's stable order), each expert's rows are cut into token tiles of
+    `tile_rows`, and the tokens of the first and the last row of every tile of every
+    touched expert are taken (so every touched expert, every full tile and every
+    ragged tail), plus `extra` random tokens.  Bookkeeping only: no layer arithmetic."""
+    ids = np.asarray(ids)
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    picked = set()
+    for e in range(E):
+        pairs = np.nonzero(flat == e)[0]          # ascending p
+        for r0 in range(0, pairs.size, tile_rows):
+            r1 = min(r0 + tile_rows, pairs.size) - 1
+            picked.add(int(pairs[r0]) // k)
+            picked.add(int(pairs[r1]) // k)
+    rng = np.random.default_rng(seed)
+    rest = np.setdiff1d(np.arange(T), np.fromiter(picked, dtype=np.int64, count=len(picked)))
+    if rest.size and extra:
+        picked.update(int(t) for t in rng.choice(rest, size=min(extra, rest.size), replace=False))
+    return np.sort(np.fromiter(picked, dtype=np.int64, count=len(picked)))

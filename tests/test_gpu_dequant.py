@@ -40,25 +40,19 @@ def test_ragged_shapes(moe_gpu, oracle_mod, E, N, K):
     assert moe_gpu.moe_get_device_error() == 0
 
 
-def test_full_gpt_oss_20b_bank_sampled_rows(moe_gpu, oracle_mod):
+def test_full_gpt_oss_20b_bank_bit_exact(moe_gpu, oracle_mod):
     # The standalone dequant workload at full size: gate_up [32, 5760, 2880] and
-    # down [32, 2880, 2880], scale bytes in [110, 130].  Every output row is
-    # produced on the GPU; rows sampled across experts are checked bit-exact, and
-    # every row's extreme values are checked against the largest possible |value|.
+    # down [32, 2880, 2880], scale bytes in [110, 130]; every element of both banks
+    # is compared with the oracle bit for bit.
     import torch
     gu, dn = make_dequant_bank(seed=0)
-    rng = np.random.default_rng(1)
     for bank in (gu, dn):
         E, N, K = bank.shape
         out = moe_gpu.mxfp4_dequantize(to_dev(bank.blocks), to_dev(bank.scales))
         torch.cuda.synchronize()
-        rows = np.concatenate([[0, E * N - 1], rng.choice(E * N, size=62, replace=False)])
-        flat_blocks = bank.blocks.reshape(E * N, K // 2)
-        flat_scales = bank.scales.reshape(E * N, K // 32)
-        want = oracle_mod.dequantize(flat_blocks[rows], flat_scales[rows], 1, len(rows), K)[0]
-        got = bits_of(out.view(E * N, K)[torch.as_tensor(rows, device=out.device)])
-        np.testing.assert_array_equal(got, want)
-        amax = out.float().abs().amax().item()
-        assert amax <= 6.0 * 2.0 ** (130 - 127) and not torch.isnan(out).any().item()
+        got = bits_of(out)
         del out
+        want = oracle_mod.dequantize(bank.blocks, bank.scales, E, N, K)
+        assert np.array_equal(got, want), f"{int(np.count_nonzero(got != want))} elements differ"
+        del got, want
     assert moe_gpu.moe_get_device_error() == 0

@@ -12,14 +12,14 @@ import numpy as np
 import pytest
 
 from mxfp4_expert_ffn_moe_b200.workloads import make_layer, make_nvfp4_dequant_bank, workload
-from tests._metrics import MAX_ABS_OVER_RMS_TOL, REL_L2_TOL, max_abs_over_rms, rel_l2
+from tests._metrics import (MAX_ABS_OVER_RMS_TOL, REL_L2_TOL, envelope_excess_over_rms,
+                            max_abs_over_rms, rel_l2)
 from tests.gpu_util import (bf16_tensor_to_f64, bits_of, nvfp4_layer_to_device, oracle_nvfp4_forward,
-                            run_nvfp4_forward, sample_tokens, to_dev)
+                            run_nvfp4_forward, sample_tokens, stratified_tokens, to_dev)
 
 pytestmark = pytest.mark.gpu
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-BF16_U2 = 2.0 ** -8
 
 
 def _gpu_dequant(moe, blocks, scales, scale2):
@@ -95,22 +95,19 @@ def test_dequant_tiny_and_huge_products_round_once(moe_gpu, oracle_mod):
     assert moe_gpu.moe_get_device_error() == 0
 
 
-def test_dequant_full_20b_bank_sampled_rows(moe_gpu, oracle_mod):
+def test_dequant_full_20b_bank_bit_exact(moe_gpu, oracle_mod):
+    # the NVFP4 twin of the gpt-oss-20b bank, every element of both projections
     import torch
     gu, dn = make_nvfp4_dequant_bank(seed=0)
-    rng = np.random.default_rng(2)
     for bank in (gu, dn):
         E, N, K = bank.shape
         out = moe_gpu.nvfp4_dequantize(to_dev(bank.blocks), to_dev(bank.scales), to_dev(bank.scale2))
         torch.cuda.synchronize()
-        rows = np.concatenate([[0, E * N - 1], rng.choice(E * N, size=62, replace=False)])
-        got = bits_of(out.view(E * N, K)[torch.as_tensor(rows, device=out.device)])
-        fb = bank.blocks.reshape(E * N, K // 2)
-        fs = bank.scales.reshape(E * N, K // 16)
-        for i, r in enumerate(rows):
-            want = oracle_mod.nvfp4_dequantize(fb[r:r + 1], fs[r:r + 1], bank.scale2[r // N:r // N + 1],
-                                               1, 1, K)[0, 0]
-            np.testing.assert_array_equal(got[i], want)
+        got = bits_of(out)
+        del out
+        want = oracle_mod.nvfp4_dequantize(bank.blocks, bank.scales, bank.scale2, E, N, K)
+        assert np.array_equal(got, want), f"{int(np.count_nonzero(got != want))} elements differ"
+        del got, want
     assert moe_gpu.moe_get_device_error() == 0
 
 
@@ -122,23 +119,22 @@ def _assert_close(got, want, what=""):
 
 
 def _assert_close_envelope(got, want, env, what=""):
-    # the bound of the MXFP4 edge tests: bf16 output rounding plus one bf16 rounding of
-    # each activation operand, scaled by the down projection's magnitude envelope
-    got = np.asarray(got, np.float64)
-    want = np.asarray(want, np.float64)
-    rms = float(np.sqrt(np.mean(want * want)))
-    excess = np.abs(got - want) - BF16_U2 * (np.abs(want) + env)
-    r = rel_l2(got, want)
-    m = float(np.max(excess)) / rms
+    """The edge-shape bound (tests/_metrics.py): bf16 output rounding plus one bf16
+    rounding of each activation operand, scaled by the magnitude envelope."""
+    r, m = rel_l2(got, want), envelope_excess_over_rms(got, want, env)
     assert r <= REL_L2_TOL and m <= MAX_ABS_OVER_RMS_TOL, f"{what}: rel_l2={r:.3g} excess/rms={m:.3g}"
 
 
-def _check_layer(moe, oracle, layer, n_sample=None, seed=0, envelope=False):
+def _check_layer(moe, oracle, layer, n_sample=None, seed=0, envelope=False, stratified=False):
     dev = nvfp4_layer_to_device(layer)
     ids, w = oracle.route(layer.logits, layer.k)
     out = run_nvfp4_forward(moe, dev, ids, w, layer)
     got = bf16_tensor_to_f64(out)
-    tokens = sample_tokens(layer.T, n_sample or layer.T, seed)
+    if stratified:
+        tile = moe.moe_token_tile_rows(layer.T, layer.H, layer.I, layer.E, layer.k, nvfp4=True)
+        tokens = stratified_tokens(ids, layer.E, tile, extra=8, seed=seed)
+    else:
+        tokens = sample_tokens(layer.T, n_sample or layer.T, seed)
     if envelope:
         want, env = oracle_nvfp4_forward(oracle, layer, ids, w, tokens, envelope=True)
         _assert_close_envelope(got[tokens], want, env, layer.name)
@@ -166,9 +162,13 @@ def test_edge_shapes(moe_gpu, oracle_mod, T, H, I, E, k, woi):
     _check_layer(moe_gpu, oracle_mod, layer, envelope=True)
 
 
-@pytest.mark.parametrize("name,n_sample", [("nvfp4_20b_decode_T8", 8), ("nvfp4_20b_prefill_T4096", 24)])
-def test_full_size_workloads_sampled(moe_gpu, oracle_mod, name, n_sample):
-    _check_layer(moe_gpu, oracle_mod, workload(name), n_sample=n_sample)
+def test_full_size_decode_every_token(moe_gpu, oracle_mod):
+    _check_layer(moe_gpu, oracle_mod, workload("nvfp4_20b_decode_T8"))
+
+
+def test_full_size_prefill_every_tile(moe_gpu, oracle_mod):
+    # every touched expert, the first and last row of each of its token tiles
+    _check_layer(moe_gpu, oracle_mod, workload("nvfp4_20b_prefill_T4096"), stratified=True)
 
 
 def test_missing_scale2_means_one(moe_gpu, oracle_mod):

@@ -92,3 +92,23 @@ def test_router_ids_only_and_bad_sizes(moe_gpu, oracle_mod):
     with pytest.raises(moe_gpu.MoEError) as ei:
         moe_gpu.moe_router_route(x, w, None, 2)
     assert ei.value.status == -1
+
+
+def test_router_nan_logits_follow_the_routing_rule(moe_gpu):
+    # a NaN router bias makes that expert's logit NaN for every token: it is never
+    # chosen; with E = k + 1 and two NaN columns every token has one empty slot
+    import torch
+    r = make_router(40, 128, 5, 4, seed=3)
+    x = to_dev(r.x_bits, torch.bfloat16)
+    w = to_dev(r.w_bits, torch.bfloat16)
+    b = r.bias.copy()
+    b[[1, 3]] = np.nan
+    moe_gpu.moe_get_device_error()
+    ids, wt, lg = moe_gpu.moe_router_route(x, w, to_dev(b), r.k, want_logits=True)
+    assert moe_gpu.moe_get_device_error() & moe_gpu.MOE_DEVERR_BAD_LOGIT
+    ids, wt = ids.cpu().numpy(), wt.cpu().numpy()
+    assert np.all(ids[:, 3] == -1) and np.all(wt[:, 3] == 0.0)
+    assert not np.isin(ids[:, :3], [1, 3]).any()
+    np.testing.assert_allclose(wt.astype(np.float64).sum(axis=1), 1.0, atol=1e-6)
+    ids2, w2 = moe_gpu.moe_route(lg, r.k)
+    assert torch.equal(ids2.cpu(), torch.from_numpy(ids)) and torch.equal(w2.cpu(), torch.from_numpy(wt))
