@@ -268,6 +268,68 @@ int moe_nvfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                          float limit, uint16_t *out, uint32_t flags, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/*
+ * Expert parallelism (transformers PR #49431 "Restore GPT-OSS's router-masked
+ * expert-parallel plan": with the experts spread over ranks, each rank's MXFP4
+ * experts consume the routing data restricted to the experts it owns).  A rank that
+ * owns experts [base, base + E_local) of the layer runs the layer in four calls
+ * around two exchanges:
+ *   moe_permute          its tokens' pairs in expert order (= owner order when
+ *                        experts are split into contiguous ranges), pair_rows given
+ *   moe_gather_pairs     the rows to ship: x rows, expert ids, routing weights
+ *   (exchange)           rows offsets[base_r] .. offsets[base_r + E_r] go to rank r
+ *   moe_mxfp4_expert_rows  the received rows through the rank's own experts -> fp32
+ *   (exchange back)      each row returns to the rank it came from, in the same order
+ *   moe_combine_pairs    the returned rows summed per token in slot order
+ * On one rank the four calls give moe_mxfp4_forward_ex's output bit for bit.
+ */
+
+/*
+ * moe_gather_pairs -- the expert-ordered rows of a permutation as a self-contained
+ * batch.  For r < offsets[E] (read on the device), p = sorted_pairs[r]:
+ *   x_rows[r] = x[p / k]   bf16 [T*k, H] (rows past offsets[E] untouched)
+ *   row_ids[r] = ids[p]    int32 [T*k]
+ *   row_weights[r] = weights[p]   fp32 [T*k]
+ * x [T, H] bf16, ids / weights [T, k]; sorted_pairs and offsets as moe_permute wrote
+ * them.  Sizes: T >= 1; 1 <= k <= 8; 1 <= E <= 256; H % 8 == 0; x and x_rows 16-byte
+ * aligned.  Errors: MOE_ERR_INVALID_ARG.
+ */
+int moe_gather_pairs(const uint16_t *x, int64_t T, int64_t H, int k, const int32_t *ids, const float *weights,
+                     const int32_t *sorted_pairs, const int32_t *offsets, int64_t E, uint16_t *x_rows,
+                     int32_t *row_ids, float *row_weights, void *stream);
+
+/*
+ * moe_mxfp4_expert_rows -- R independent rows through the experts of a bank slice:
+ * row r goes to expert row_ids[r] - expert_base of gate_up_* / down_* (banks of E
+ * experts, laid out as for moe_mxfp4_forward_ex) and
+ *   y_rows[r] = row_weights[r] * (W_d a + b_d)      (flags 0: weight on the output)
+ *   y_rows[r] = W_d a                               (MOE_FLAG_WEIGHT_ON_INPUT: the
+ *                                                    expert input is bf16(w * x))
+ * with a the clamped SwiGLU of W_gu x + b_gu, i.e. one slot of moe_mxfp4_forward_ex
+ * before the combine, in fp32 [R, H] (16-byte aligned).  Rows whose id falls outside
+ * [expert_base, expert_base + E) are left unwritten and raise
+ * MOE_DEVERR_BAD_EXPERT_ID.  workspace: NULL (allocated stream-ordered) or at least
+ * moe_mxfp4_workspace_size(R, H, I, E, 1) bytes.  Every other rule and error as
+ * moe_mxfp4_forward_ex; expert_base must lie in [0, 2^31).
+ */
+int moe_mxfp4_expert_rows(const uint16_t *x_rows, int64_t R, int64_t H, int64_t I, int64_t E, int64_t expert_base,
+                          const int32_t *row_ids, const float *row_weights, const uint8_t *gate_up_blocks,
+                          const uint8_t *gate_up_scales, const float *gate_up_bias,
+                          const uint8_t *down_blocks, const uint8_t *down_scales, const float *down_bias,
+                          float alpha, float limit, float *y_rows, uint32_t flags, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/*
+ * moe_combine_pairs -- out[t] = sum over j < k of y_rows[pair_rows[t*k + j]] in slot
+ * order, in fp32, rounded once to bf16; slots whose pair_rows entry is -1 contribute
+ * nothing (FreeToken PR #838 review: the result is sum w*(y + b), the weight already
+ * inside each row).  y_rows fp32 [rows, H] (16-byte aligned), pair_rows int32
+ * [T*k] (moe_permute's inverse), out bf16 [T, H].  Sizes: T >= 1; 1 <= k <= 8;
+ * H % 4 == 0.  Errors: MOE_ERR_INVALID_ARG.
+ */
+int moe_combine_pairs(const float *y_rows, const int32_t *pair_rows, int64_t T, int k, int64_t H, uint16_t *out,
+                      void *stream);
+
 /* Static English text for a moe_status value. */
 const char *moe_status_string(int status);
 

@@ -23,7 +23,8 @@ __all__ = [
     "moe_mxfp4_forward_noalloc", "MOE_NOALLOC_SCRATCH_BYTES",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
     "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host", "moe_permute", "moe_token_tile_rows",
-    "MOE_DEVERR_BAD_LOGIT", "MOE_DEVERR_OUT_OF_BOUNDS",
+    "MOE_DEVERR_BAD_LOGIT", "MOE_DEVERR_OUT_OF_BOUNDS", "use_checked_library", "moe_gather_pairs", "moe_mxfp4_expert_rows",
+    "moe_combine_pairs",
 ]
 
 MOE_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
@@ -41,11 +42,14 @@ EXPORTED_SYMBOLS = (
     "moe_profile_enable", "moe_profile_enable_stages", "moe_profile_read", "moe_mxfp4_forward_noalloc",
     "nvfp4_dequantize", "moe_nvfp4_forward_ex", "moe_router_route",
     "mxfp4_dequantize_from_host", "nvfp4_dequantize_from_host", "moe_permute", "moe_token_tile_rows",
+    "moe_gather_pairs", "moe_mxfp4_expert_rows", "moe_combine_pairs",
 )
 PROFILE_STAGES = ("route", "permute", "gather", "gate_up", "down", "combine", "dequant")
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _lib = None
+_libs = {}
+_use_checked = False
 
 
 class MoEError(RuntimeError):
@@ -54,16 +58,32 @@ class MoEError(RuntimeError):
         self.status = status
 
 
-def library_path() -> str:
-    return os.path.join(_PKG, "libmoe_mxfp4.so")
+def library_path(checked: bool = False) -> str:
+    return os.path.join(_PKG, "libmoe_mxfp4_checked.so" if checked else "libmoe_mxfp4.so")
+
+
+def use_checked_library(on: bool) -> bool:
+    """Route every call of this binding to the bounds-checked build of the library
+    (built by build.build(checked=True); each data-dependent global index is tested
+    and MOE_DEVERR_OUT_OF_BOUNDS raised instead of an access outside a buffer), or
+    back to the normal build.  Returns the previous setting."""
+    global _use_checked, _lib
+    prev = _use_checked
+    _use_checked = bool(on)
+    _lib = None
+    return prev
 
 
 def load_library():
-    """Load the in-tree CUDA library; raise if it has not been built."""
+    """Load the in-tree CUDA library (the variant use_checked_library selects); raise if
+    it has not been built."""
     global _lib
     if _lib is not None:
         return _lib
-    path = library_path()
+    path = library_path(_use_checked)
+    if path in _libs:
+        _lib = _libs[path]
+        return _lib
     if not os.path.exists(path):
         raise RuntimeError(f"CUDA library not built: {path} (run __graft_entry__.build())")
     lib = ctypes.CDLL(path)
@@ -105,8 +125,16 @@ def load_library():
     lib.moe_permute.restype = i32
     lib.moe_token_tile_rows.argtypes = [i64, i64, i64, i64, i32, i32]
     lib.moe_token_tile_rows.restype = i32
+    lib.moe_gather_pairs.argtypes = [p, i64, i64, i32, p, p, p, p, i64, p, p, p, p]
+    lib.moe_gather_pairs.restype = i32
+    lib.moe_mxfp4_expert_rows.argtypes = [p, i64, i64, i64, i64, i64, p, p, p, p, p, p, p, p, f32, f32, p,
+                                          ctypes.c_uint32, p, ctypes.c_size_t, p]
+    lib.moe_mxfp4_expert_rows.restype = i32
+    lib.moe_combine_pairs.argtypes = [p, p, i64, i32, i64, p, p]
+    lib.moe_combine_pairs.restype = i32
     lib.moe_profile_read.argtypes = [p, p]
     lib.moe_profile_read.restype = i32
+    _libs[path] = lib
     _lib = lib
     return lib
 
@@ -341,6 +369,62 @@ def moe_permute(ids, E: int, tile_rows: int, want_pair_rows: bool = True, stream
         *[_dev(out[n], torch.int32, n) for n in ("counts", "offsets", "tile_offsets", "sorted_pairs")],
         _dev(out.get("pair_rows"), torch.int32, "pair_rows"), _stream(stream))
     _check("moe_permute", rc)
+    return out
+
+
+def moe_gather_pairs(x, ids, weights, perm, E: int, stream=None):
+    """Rows of x in the expert order of `perm` (moe_permute's dict), with their expert
+    ids and routing weights: (bf16 [T*k, H], int32 [T*k], fp32 [T*k]); only the first
+    perm["offsets"][E] rows are written."""
+    import torch
+    T, H = x.shape
+    k = ids.shape[1]
+    x_rows = torch.empty((T * k, H), dtype=torch.bfloat16, device=x.device)
+    row_ids = torch.empty(T * k, dtype=torch.int32, device=x.device)
+    row_w = torch.empty(T * k, dtype=torch.float32, device=x.device)
+    rc = load_library().moe_gather_pairs(
+        _dev(x, torch.bfloat16, "x"), T, H, int(k), _dev(ids, torch.int32, "ids"),
+        _dev(weights, torch.float32, "weights"), _dev(perm["sorted_pairs"], torch.int32, "sorted_pairs"),
+        _dev(perm["offsets"], torch.int32, "offsets"), int(E), _dev(x_rows, torch.bfloat16, "x_rows"),
+        _dev(row_ids, torch.int32, "row_ids"), _dev(row_w, torch.float32, "row_weights"), _stream(stream))
+    _check("moe_gather_pairs", rc)
+    return x_rows, row_ids, row_w
+
+
+def moe_mxfp4_expert_rows(x_rows, row_ids, row_weights, expert_base: int, gate_up_blocks, gate_up_scales,
+                          gate_up_bias, down_blocks, down_scales, down_bias, alpha: float = 1.702,
+                          limit: float = 7.0, flags: int = 0, y_rows=None, workspace=None, stream=None):
+    """Rows x_rows [R, H] through experts row_ids - expert_base of the given banks ->
+    fp32 [R, H] (one weighted slot of the layer per row, no combine)."""
+    import torch
+    R, H = x_rows.shape
+    E, N2, _ = gate_up_blocks.shape
+    if y_rows is None:
+        y_rows = torch.empty((R, H), dtype=torch.float32, device=x_rows.device)
+    ws = _dev(workspace, torch.uint8, "workspace")
+    nbytes = 0 if workspace is None else workspace.numel()
+    rc = load_library().moe_mxfp4_expert_rows(
+        _dev(x_rows, torch.bfloat16, "x_rows"), R, H, N2 // 2, E, int(expert_base),
+        _dev(row_ids, torch.int32, "row_ids"), _dev(row_weights, torch.float32, "row_weights"),
+        _dev(gate_up_blocks, torch.uint8, "gate_up_blocks"), _dev(gate_up_scales, torch.uint8, "gate_up_scales"),
+        _dev(gate_up_bias, torch.float32, "gate_up_bias"), _dev(down_blocks, torch.uint8, "down_blocks"),
+        _dev(down_scales, torch.uint8, "down_scales"), _dev(down_bias, torch.float32, "down_bias"),
+        float(alpha), float(limit), _dev(y_rows, torch.float32, "y_rows"), ctypes.c_uint32(flags), ws, nbytes,
+        _stream(stream))
+    _check("moe_mxfp4_expert_rows", rc)
+    return y_rows
+
+
+def moe_combine_pairs(y_rows, pair_rows, T: int, k: int, out=None, stream=None):
+    """out[t] = sum_j y_rows[pair_rows[t*k + j]] (fp32 sum in slot order, bf16 out)."""
+    import torch
+    H = y_rows.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y_rows.device)
+    rc = load_library().moe_combine_pairs(_dev(y_rows, torch.float32, "y_rows"),
+                                          _dev(pair_rows, torch.int32, "pair_rows"), int(T), int(k), H,
+                                          _dev(out, torch.bfloat16, "out"), _stream(stream))
+    _check("moe_combine_pairs", rc)
     return out
 
 

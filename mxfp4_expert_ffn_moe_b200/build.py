@@ -9,6 +9,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_mxfp4.so")
+# the bounds-checked debugging variant (every data-dependent global index tested)
+LIB_CHECKED = os.path.join(PKG, "libmoe_mxfp4_checked.so")
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared", "-Xptxas", "-warn-spills"]
 
@@ -22,25 +24,28 @@ def _deps():
         os.path.join(os.path.dirname(PKG), "include", "moe_mxfp4.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(checked: bool = False) -> bool:
+    lib = LIB_CHECKED if checked else LIB
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Compile the library (or, with checked, its bounds-checked variant) in-tree."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(checked):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
     if os.path.exists("/usr/local/cuda/bin/nvcc") and nvcc == "nvcc":
         nvcc = "/usr/local/cuda/bin/nvcc"
-    cmd = [nvcc] + NVCC_FLAGS + _sources() + ["-o", LIB]
+    cmd = [nvcc] + NVCC_FLAGS + (["-DMOE_CHECKED=1"] if checked else []) + _sources() + ["-o", lib]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv)

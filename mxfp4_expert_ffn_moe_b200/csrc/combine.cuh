@@ -39,4 +39,35 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const float *__restri
     }
 }
 
+// out[t] = sum_{j < k} y_rows[pair_rows[t*k + j]] in slot order (fp32, one bf16
+// rounding), skipping pairs whose row is -1 (dropped): the combine of rows that come
+// back in expert order, e.g. from the ranks that own their experts.
+__global__ void __launch_bounds__(256) combine_pair_rows_kernel(const float *__restrict__ y_rows,
+                                                                const int32_t *__restrict__ pair_rows,
+                                                                int64_t T, int k, int64_t H,
+                                                                uint16_t *__restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t q = H / 4;
+    const int64_t n = T * q;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = i / q, c = i - t * q;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const int r = __ldg(pair_rows + t * k + j);
+            if (r < 0 || !in_bounds(r, T * k)) continue;
+            const float4 v = __ldcs(reinterpret_cast<const float4 *>(y_rows + (int64_t)r * H) + c);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(s.x, s.y);
+        o.y = pack_bf16x2(s.z, s.w);
+        reinterpret_cast<uint2 *>(out + t * H)[c] = o;
+    }
+}
+
 }  // namespace moe

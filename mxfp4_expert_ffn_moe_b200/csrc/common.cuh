@@ -18,6 +18,33 @@ __device__ int g_device_error;
 
 __device__ __forceinline__ void raise_device_error(int bits) { atomicOr(&g_device_error, bits); }
 
+// Bounds-checked builds (MOE_CHECKED=1, a debugging variant of the library): every
+// data-dependent global index is tested against its buffer's extent before the
+// access; an index outside [0, n) raises MOE_DEVERR_OUT_OF_BOUNDS and the access is
+// skipped (never a trap).  In the normal build the test is compiled away.
+#ifndef MOE_CHECKED
+#define MOE_CHECKED 0
+#endif
+__device__ __forceinline__ bool in_bounds(int64_t idx, int64_t n) {
+    if constexpr (MOE_CHECKED) {
+        if (idx < 0 || idx >= n) {
+            raise_device_error(MOE_DEVERR_OUT_OF_BOUNDS);
+            return false;
+        }
+    }
+    return true;
+}
+// [lo, hi) within [0, n)
+__device__ __forceinline__ bool range_in_bounds(int64_t lo, int64_t hi, int64_t n) {
+    if constexpr (MOE_CHECKED) {
+        if (lo < 0 || hi > n || lo > hi) {
+            raise_device_error(MOE_DEVERR_OUT_OF_BOUNDS);
+            return false;
+        }
+    }
+    return true;
+}
+
 // fp32 value of an E8M0 scale byte: 2^(s - 127).  s = 0 is the fp32 subnormal
 // 2^-127; s = 0xff is not a number (invalid per the MXFP4 validation rules).
 __device__ __forceinline__ float e8m0_to_f32(uint32_t s) {

@@ -180,6 +180,9 @@ __device__ __forceinline__ Tile decode_tile(const Params &p, int item, int w_til
     t.h = (t.ntok + 15) & ~15;
     t.m0 = wt * BM;
     t.mrows = min(BM, p.N - t.m0);
+    // bounds-checked builds report an inconsistent schedule (the stores below are checked)
+    range_in_bounds(t.row0, (int64_t)t.row0 + t.ntok, p.P);
+    in_bounds(t.e, p.E);
     return t;
 }
 
@@ -446,7 +449,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                     const int I = p.N / 2;
                     const int64_t RS = split_row_bytes(I);
                     const int f0 = (t.m0 >> 1) + 16 * q;     // first feature of this warp
-                    if (lane < nvalid && f0 < I) {
+                    if (lane < nvalid && f0 < I && in_bounds(t.row0 + c0 + lane, p.P) &&
+                        range_in_bounds(f0, f0 + 16, I)) {
                         const int64_t row = t.row0 + c0 + lane;
                         uint8_t *hrow = p.actq + row * RS;
                         uint8_t *lrow = p.actq + ((int64_t)p.P + row) * RS;
@@ -465,7 +469,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                     // so that each pair's row segment leaves as 16-byte stores
                     int pair_l = 0;
                     float wt_l = 1.0f;
-                    if (lane < nvalid) {
+                    if (lane < nvalid && in_bounds(t.row0 + c0 + lane, p.P)) {
                         pair_l = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
                         if (!p.weight_on_input) wt_l = __ldg(p.weights + pair_l);
                     }
@@ -485,7 +489,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                                 const int piece = rd * 32 + lane;    // 16 tokens x 8 pieces of 16 B
                                 const int tok = 16 * hf + (piece >> 3), part = piece & 7;
                                 const int pi = __shfl_sync(0xFFFFFFFFu, pair_l, tok);
-                                if (tok < nvalid) {
+                                if (tok < nvalid && in_bounds(pi, p.P) &&
+                                    range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
                                     const float4 val = *reinterpret_cast<const float4 *>(stg + (piece >> 3) * 32 + part * 4);
                                     *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
                                 }

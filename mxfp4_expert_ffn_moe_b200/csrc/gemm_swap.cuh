@@ -113,6 +113,7 @@ struct Params {
     const float *bias;            // [E, N] or null
     const float *scale2;          // NVFP4 weight_scale_2: gate_up [E, 2] (gate, up), down [E]; or null
     int E, N, K;
+    int rows_cap;                 // rows of the A, act and yp buffers (bounds-checked builds)
     // gate_up epilogue
     uint16_t *act;                // [rows, N/2] bf16
     float alpha, limit;
@@ -156,6 +157,9 @@ __device__ __forceinline__ Tile decode_tile(const Params &p, int item, int w_til
     t.ntok = min(TOK, __ldg(p.counts + t.e) - tt * TOK);
     t.m0 = wt * BM;
     t.mrows = min(BM, p.N - t.m0);
+    // bounds-checked builds report an inconsistent schedule (the stores below are checked)
+    range_in_bounds(t.row0, (int64_t)t.row0 + t.ntok, p.rows_cap);
+    in_bounds(t.e, p.E);
     return t;
 }
 
@@ -336,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < TOK / 32; ++j) {
                     const int tok = 32 * j + lane;
-                    pairs[j] = tok < t.ntok ? __ldg(p.sorted_pairs + t.row0 + tok) : 0;
+                    pairs[j] = (tok < t.ntok && in_bounds(t.row0 + tok, p.rows_cap)) ? __ldg(p.sorted_pairs + t.row0 + tok) : 0;
                     wts[j] = (tok < t.ntok && !p.weight_on_input) ? __ldg(p.weights + pairs[j]) : 1.0f;
                 }
             }
@@ -373,7 +377,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int h = 0; h < 2; ++h) {
                         const int piece = lane + 32 * h;            // 64 pieces of 16 bytes
                         const int tok = piece >> 1;
-                        if (tok < nvalid) {
+                        if (tok < nvalid && in_bounds(t.row0 + c0 + tok, p.rows_cap) &&
+                            range_in_bounds(fbase + (piece & 1) * 8, fbase + (piece & 1) * 8 + 8, p.N / 2)) {
                             const uint4 val = *reinterpret_cast<const uint4 *>(stg + tok * 16 + (piece & 1) * 8);
                             *reinterpret_cast<uint4 *>(p.act + (int64_t)(t.row0 + c0 + tok) * (p.N / 2) +
                                                        fbase + (piece & 1) * 8) = val;
@@ -413,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int piece = rd * 32 + lane;    // 32 tokens x 8 pieces of 16 B
                             const int tok = piece >> 3, part = piece & 7;
                             const int pi = __shfl_sync(0xFFFFFFFFu, pairs[c0 >> 5], tok);
-                            if (tok < nvalid) {
+                            if (tok < nvalid && in_bounds(pi, p.rows_cap) &&
+                                range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
                                 const float4 val = *reinterpret_cast<const float4 *>(stg + tok * 32 + part * 4);
                                 *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
                             }

@@ -251,6 +251,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     p.sorted_pairs = sorted_pairs;
     p.weights = weights;
     p.weight_on_input = woi;
+    p.rows_cap = (int)rows;
     const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
     auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp, kNv>;
@@ -397,35 +398,42 @@ int config_tok(TileConfig c) {
 // Pair permutation (one CTA).  The ids are staged in shared memory when they fit (up
 // to ~50K pairs); the attribute is per device, so it is set on every call, like the
 // GEMMs'.
-int launch_permute(const int32_t *ids, int64_t P, int64_t E, int tile_rows, int32_t *counts, int32_t *offsets,
-                   int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows, cudaStream_t s) {
+int launch_permute(const int32_t *ids, int expert_base, int64_t P, int64_t E, int tile_rows, int32_t *counts,
+                   int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
+                   cudaStream_t s) {
     const bool perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)moe::kPermuteSmemCap) == cudaSuccess;
     if (!perm_attr) cudaGetLastError();
     const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
     const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
     StageScope sp(MOE_STAGE_PERMUTE, s);
-    launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, P, (int)E,
-               tile_rows, staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs, pair_rows);
+    launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, expert_base, P,
+               (int)E, tile_rows, staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs, pair_rows);
     return launch_check();
 }
 
 // The whole layer on the caller's stream: permute -> gather (or split) -> gate_up ->
 // down -> combine.  nv: NVFP4 banks (E4M3 scales per 16 elements, weight_scale_2).
+// expert_base: ids are taken relative to it (the banks hold experts expert_base ..
+// expert_base + E - 1).  rows_out: when given, the weighted expert rows (fp32 [T*k, H],
+// indexed by pair) are written there and the combine is skipped (out unused).
 int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_t E, int k,
                   const int32_t *ids, const float *weights, const uint8_t *gate_up_blocks,
                   const uint8_t *gate_up_scales, const float *gate_up_scale2, const float *gate_up_bias,
                   const uint8_t *down_blocks, const uint8_t *down_scales, const float *down_scale2,
                   const float *down_bias, float alpha, float limit, uint16_t *out, uint32_t flags,
-                  void *workspace, size_t workspace_bytes, void *stream) {
+                  void *workspace, size_t workspace_bytes, void *stream, int64_t expert_base = 0,
+                  float *rows_out = nullptr) {
     if (!x || !ids || !weights || !gate_up_blocks || !gate_up_scales || !down_blocks ||
-        !down_scales || !out)
+        !down_scales || (!out && !rows_out))
         return MOE_ERR_INVALID_ARG;
+    if (expert_base < 0 || expert_base > (int64_t)0x7FFFFFFF) return MOE_ERR_INVALID_ARG;
+    if (rows_out && !aligned(rows_out, 16)) return MOE_ERR_INVALID_ARG;
     if (!forward_sizes_ok(T, H, I, E, k)) return MOE_ERR_INVALID_ARG;
     if (flags & ~MOE_FLAG_WEIGHT_ON_INPUT) return MOE_ERR_INVALID_ARG;
     const bool woi = (flags & MOE_FLAG_WEIGHT_ON_INPUT) != 0;
     if (woi && (gate_up_bias || down_bias)) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(gate_up_blocks, 16) ||
+    if (!aligned(x, 16) || (out && !aligned(out, 16)) || !aligned(gate_up_blocks, 16) ||
         !aligned(down_blocks, 16) || !aligned(gate_up_scales, 16) || !aligned(down_scales, 16) ||
         !aligned(ids, 4) || !aligned(weights, 4) ||
         !aligned(gate_up_bias, 4) || !aligned(down_bias, 4) ||
@@ -452,14 +460,14 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     int32_t *sorted_pairs = reinterpret_cast<int32_t *>(ws + L.sorted_pairs);
     uint16_t *x_perm = reinterpret_cast<uint16_t *>(ws + L.x_perm);
     uint16_t *act = reinterpret_cast<uint16_t *>(ws + L.act);
-    float *yp = reinterpret_cast<float *>(ws + L.yp);
+    float *yp = rows_out ? rows_out : reinterpret_cast<float *>(ws + L.yp);
 
     const int64_t P = T * k;
     const TileConfig cfg = pick_config(P, H, I, E, nv);
     int rc = MOE_OK;
     do {
-        if ((rc = launch_permute(ids, P, E, config_tok(cfg), counts, offsets, tile_offsets, sorted_pairs,
-                                 nullptr, s)) != MOE_OK)
+        if ((rc = launch_permute(ids, (int)expert_base, P, E, config_tok(cfg), counts, offsets, tile_offsets,
+                                 sorted_pairs, nullptr, s)) != MOE_OK)
             break;
         const bool mxf = cfg == kDecodeMxf || cfg == kPrefillMxf;
         if (mxf) {
@@ -478,7 +486,8 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
                     moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
                 StageScope sg(MOE_STAGE_GATHER, s);
                 launch_pdl(moe::gather_rows_kernel, dim3((unsigned)gather_grid), dim3(256), 0, s, x, weights,
-                           sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm);
+                           sorted_pairs, offsets, (int)E, k, H, woi ? 1 : 0, x_perm, nullptr, nullptr,
+                           nullptr, P);
             }
             if ((rc = launch_check()) != MOE_OK) break;
 #define MOE_PROJECTIONS(C, NV)                                                                    \
@@ -494,7 +503,7 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
                                         : MOE_PROJECTIONS(moe::swp::PrefillCfg, false);
 #undef MOE_PROJECTIONS
         }
-        if (rc != MOE_OK) break;
+        if (rc != MOE_OK || rows_out) break;
         {
             const int64_t n4 = T * (H / 4);
             const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;
@@ -685,13 +694,56 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
     return launch_check();
 }
 
+int moe_gather_pairs(const uint16_t *x, int64_t T, int64_t H, int k, const int32_t *ids, const float *weights,
+                     const int32_t *sorted_pairs, const int32_t *offsets, int64_t E, uint16_t *x_rows,
+                     int32_t *row_ids, float *row_weights, void *stream) {
+    if (!x || !ids || !weights || !sorted_pairs || !offsets || !x_rows || !row_ids || !row_weights)
+        return MOE_ERR_INVALID_ARG;
+    if (T < 1 || k < 1 || k > 8 || E < 1 || E > 256 || H < 8 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_rows, 16)) return MOE_ERR_INVALID_ARG;
+    const int64_t P = T * k;
+    const int64_t grid = moe::ceil_div(P, 8) < sm_count() * 8 ? moe::ceil_div(P, 8) : sm_count() * 8;
+    cudaStream_t s = (cudaStream_t)stream;
+    StageScope sg(MOE_STAGE_GATHER, s);
+    launch_pdl(moe::gather_rows_kernel, dim3((unsigned)grid), dim3(256), 0, s, x, weights, sorted_pairs, offsets,
+               (int)E, k, H, 0, x_rows, ids, row_ids, row_weights, P);
+    return launch_check();
+}
+
+int moe_mxfp4_expert_rows(const uint16_t *x_rows, int64_t R, int64_t H, int64_t I, int64_t E, int64_t expert_base,
+                          const int32_t *row_ids, const float *row_weights, const uint8_t *gate_up_blocks,
+                          const uint8_t *gate_up_scales, const float *gate_up_bias,
+                          const uint8_t *down_blocks, const uint8_t *down_scales, const float *down_bias,
+                          float alpha, float limit, float *y_rows, uint32_t flags, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+    if (!y_rows) return MOE_ERR_INVALID_ARG;
+    return forward_layer(false, x_rows, R, H, I, E, 1, row_ids, row_weights, gate_up_blocks, gate_up_scales,
+                         nullptr, gate_up_bias, down_blocks, down_scales, nullptr, down_bias, alpha, limit,
+                         nullptr, flags, workspace, workspace_bytes, stream, expert_base, y_rows);
+}
+
+int moe_combine_pairs(const float *y_rows, const int32_t *pair_rows, int64_t T, int k, int64_t H, uint16_t *out,
+                      void *stream) {
+    if (!y_rows || !pair_rows || !out) return MOE_ERR_INVALID_ARG;
+    if (T < 1 || k < 1 || k > 8 || H < 4 || H % 4 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned(y_rows, 16) || !aligned(out, 8)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t n4 = T * (H / 4);
+    const int64_t cgrid = moe::ceil_div(n4, 256) < sm_count() * 16 ? moe::ceil_div(n4, 256) : sm_count() * 16;
+    StageScope sc(MOE_STAGE_COMBINE, s);
+    launch_pdl(moe::combine_pair_rows_kernel, dim3((unsigned)cgrid), dim3(256), 0, s, y_rows, pair_rows, T, k, H,
+               out);
+    return launch_check();
+}
+
 int moe_permute(const int32_t *ids, int64_t T, int k, int64_t E, int tile_rows, int32_t *counts,
                 int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
                 void *stream) {
     if (!ids || !counts || !offsets || !tile_offsets || !sorted_pairs) return MOE_ERR_INVALID_ARG;
     if (T < 1 || k < 1 || k > 8 || E < 1 || E > 256 || tile_rows < 1) return MOE_ERR_INVALID_ARG;
     if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
-    return launch_permute(ids, T * k, E, tile_rows, counts, offsets, tile_offsets, sorted_pairs, pair_rows,
+    return launch_permute(ids, 0, T * k, E, tile_rows, counts, offsets, tile_offsets, sorted_pairs, pair_rows,
                           (cudaStream_t)stream);
 }
 

@@ -31,8 +31,16 @@ __host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t P, bool s
 }
 constexpr size_t kPermuteSmemCap = 200 * 1024;
 
+__device__ __forceinline__ int relative_expert(int32_t id, int expert_base, int E) {
+    const int64_t e = (int64_t)id - expert_base;
+    return (e >= 0 && e < E) ? (int)e : -1;
+}
+
+// ids are taken relative to expert_base: pair p belongs to expert ids[p] - expert_base
+// of the E experts handled here (a rank's slice of the experts under expert parallelism;
+// 0 for the whole layer).
 __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
-    const int32_t *__restrict__ ids, int64_t P, int E, int bm, int staged, int32_t *__restrict__ counts,
+    const int32_t *__restrict__ ids, int expert_base, int64_t P, int E, int bm, int staged, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
     int32_t *__restrict__ sorted_pairs, int32_t *__restrict__ pair_rows) {
     pdl_wait();
@@ -44,15 +52,16 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
     if (staged)
-        for (int64_t i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = __ldg(ids + i);
+        for (int64_t i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = relative_expert(__ldg(ids + i), expert_base, E);
     __syncthreads();
-    const int32_t *src = staged ? ids_s : ids;
+    // expert of pair p relative to expert_base, -1 when outside [0, E)
+    auto expert_of = [&](int64_t p) { return staged ? ids_s[p] : relative_expert(__ldg(ids + p), expert_base, E); };
 
     const int64_t chunk = (P + 31) / 32;
     const int64_t beg = (int64_t)warp * chunk;
     const int64_t end = (beg + chunk < P) ? beg + chunk : P;
     for (int64_t p = beg + lane; p < end; p += 32) {
-        const int e = src[p];
+        const int e = expert_of(p);
         if ((unsigned)e < (unsigned)E)
             atomicAdd(&cnt[warp * E + e], 1);
         else
@@ -87,14 +96,14 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     __syncthreads();
     for (int64_t base = beg; base < end; base += 32) {
         const int64_t p = base + lane;
-        const int e = (p < end) ? src[p] : -1;
+        const int e = (p < end) ? expert_of(p) : -1;
         const bool valid = (p < end) && (unsigned)e < (unsigned)E;
         const int key = valid ? e : -1 - lane;
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
         const int rank = __popc(peers & ((1u << lane) - 1u));
         const int wbase = valid ? cnt[warp * E + e] : 0;
         __syncwarp();
-        if (valid) {
+        if (valid && in_bounds(off[e] + wbase + rank, P)) {
             sorted_pairs[off[e] + wbase + rank] = (int32_t)p;
             if (rank == 0) cnt[warp * E + e] = wbase + __popc(peers);
         }
@@ -105,10 +114,14 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
 
 // x_perm[r] = x[t] (router weight on the output) or bf16(w[p] * x[t]) (router
 // weight on the input), t = sorted_pairs[r] / k.  One warp per row, 16-byte chunks.
+// Optionally (row_ids / row_weights non-null) also row_ids[r] = ids[p] and
+// row_weights[r] = weights[p]: the rows as a self-contained batch, e.g. to ship to the
+// rank that owns their experts.
 __global__ void __launch_bounds__(256) gather_rows_kernel(
     const uint16_t *__restrict__ x, const float *__restrict__ weights,
     const int32_t *__restrict__ sorted_pairs, const int32_t *__restrict__ offsets, int E, int k,
-    int64_t H, int weight_on_input, uint16_t *__restrict__ x_perm) {
+    int64_t H, int weight_on_input, uint16_t *__restrict__ x_perm, const int32_t *__restrict__ ids,
+    int32_t *__restrict__ row_ids, float *__restrict__ row_weights, int64_t P) {
     pdl_wait();
     pdl_trigger();
     const int rows = offsets[E];
@@ -118,10 +131,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
     for (int64_t r = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); r < rows;
          r += (int64_t)gridDim.x * wpb) {
         const int p = sorted_pairs[r];
+        if (!in_bounds(r, P) || !in_bounds(p, P)) continue;   // warp-uniform (one row per warp)
         const int64_t t = p / k;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(x_perm + r * H);
         const float w = weight_on_input ? weights[p] : 1.0f;
+        if (lane == 0 && row_ids) row_ids[r] = ids[p];
+        if (lane == 0 && row_weights) row_weights[r] = weights[p];
         // four 16-byte loads in flight per lane before their stores
         for (int64_t c0 = lane; c0 < chunks; c0 += 4 * 32) {
             uint4 v[4];

@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(256) split_rows_kernel(
         const int64_t r = it / steps;
         const int64_t st = it - r * steps;
         const int p = __ldg(sorted_pairs + r);
+        if (!in_bounds(r, P) || !in_bounds(p, P)) continue;   // warp-uniform (one item per warp)
         const int64_t c = st * 128 + 4 * lane;
         const bool in = c < K;                               // K is a multiple of 32
         uint2 raw = make_uint2(0u, 0u);

@@ -85,12 +85,15 @@ def make_bank(rng: np.random.Generator, E: int, N: int, K: int, scale_lo: int,
 def make_layer(T: int, H: int, I: int, E: int, k: int, seed: int = 0, scale_lo: int = 118,
                scale_hi: int = 126, zipf: float = 0.0, biases: bool = True,
                weight_on_input: bool = False, bias_std: float = 0.02,
-               name: str = "", fmt: str = "mxfp4") -> MoELayer:
-    assert fmt in ("mxfp4", "nvfp4")
+               name: str = "", fmt: str = "mxfp4", x_dist: str = "normal") -> MoELayer:
+    assert fmt in ("mxfp4", "nvfp4") and x_dist in ("normal", "wide")
     if fmt == "nvfp4":
         return _make_nvfp4_layer(T, H, I, E, k, seed, zipf, biases, weight_on_input, bias_std, name)
     rng = np.random.default_rng(seed)
-    x_bits = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    if x_dist == "wide":
+        x_bits = _wide_range_rows(rng, T, H)
+    else:
+        x_bits = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
     logits = rng.standard_normal((T, E), dtype=np.float32)
     if zipf:
         rank = np.arange(1, E + 1, dtype=np.float64)
@@ -104,6 +107,20 @@ def make_layer(T: int, H: int, I: int, E: int, k: int, seed: int = 0, scale_lo: 
         d_bias = None
     return MoELayer(T, H, I, E, k, x_bits, logits, gu, gu_bias, dn, d_bias,
                     weight_on_input=weight_on_input, name=name)
+
+
+def _wide_range_rows(rng: np.random.Generator, T: int, H: int) -> np.ndarray:
+    """bf16 rows whose 32-element blocks each hold one large element (magnitude
+    2^u, u uniform in [0, 3)) at a random position and 31 smaller ones spread
+    log-uniformly from it down to 2^-20 of it, random signs."""
+    nb = H // 32
+    big = 2.0 ** rng.uniform(0.0, 3.0, size=(T, nb, 1))
+    below = rng.uniform(0.0, 20.0, size=(T, nb, 32))
+    pos = rng.integers(0, 32, size=(T, nb))
+    np.put_along_axis(below, pos[..., None], 0.0, axis=2)
+    sign = np.where(rng.integers(0, 2, size=(T, nb, 32)) == 1, -1.0, 1.0)
+    x = (sign * big * 2.0 ** (-below)).reshape(T, H).astype(np.float32)
+    return f32_to_bf16_bits(x)
 
 
 def _make_nvfp4_layer(T, H, I, E, k, seed, zipf, biases, weight_on_input, bias_std, name):
@@ -158,6 +175,12 @@ WORKLOADS = {
     "20b_prefill_T4096": dict(T=4096, H=2880, I=2880, E=32, k=4),
     "120b_zipf_T256": dict(T=256, H=2880, I=2880, E=128, k=4, zipf=1.5),
     "120b_zipf_T8192": dict(T=8192, H=2880, I=2880, E=128, k=4, zipf=1.5),
+    # test cases only: activation blocks spanning 2^20 (one large element, the rest
+    # down to 2^-20 of it) and heavy gate_up biases (gate values far below zero give
+    # activations near zero beside large ones), the hardest inputs for an operand
+    # kept as a few significant bits per block scale
+    "tiny_wide": dict(T=16, H=256, I=256, E=4, k=2, x_dist="wide", bias_std=3.0),
+    "20b_decode_wide_T8": dict(T=8, H=2880, I=2880, E=32, k=4, x_dist="wide", bias_std=3.0),
     # the NVFP4 expert variant of the same layers
     "nvfp4_tiny_woo": dict(T=8, H=128, I=128, E=4, k=2, biases=True, fmt="nvfp4"),
     "nvfp4_tiny_woi": dict(T=8, H=128, I=128, E=4, k=2, biases=False, weight_on_input=True,

@@ -50,6 +50,7 @@ DEFECT_DOWN_BIAS_IN_SCALE = 8
 DEFECT_NVFP4_SCALE_AFTER_BIAS = 9
 DEFECT_NVFP4_BLOCK32 = 10
 DEFECT_NVFP4_GU_SCALE_SWAP = 11
+DEFECT_OPERAND_E4M3_HI_ONLY = 12
 
 FLAG_WEIGHT_ON_INPUT = 1
 

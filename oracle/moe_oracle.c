@@ -86,6 +86,12 @@ enum {
                                                first 16-block's scale for both halves) */
     ORACLE_DEFECT_NVFP4_GU_SCALE_SWAP = 11, /* NVFP4: gate rows take the up scale and
                                                the other way round                    */
+    ORACLE_DEFECT_OPERAND_E4M3_HI_ONLY = 12, /* both projections' activation operands
+                                               kept to one E4M3 term per element at a
+                                               power-of-two scale per 32-element block
+                                               (2^(e-7), e the exponent of the block's
+                                               largest magnitude): a kernel that drops
+                                               the second term of a two-term split    */
 };
 
 enum { ORACLE_FMT_MXFP4 = 0, ORACLE_FMT_NVFP4 = 1 };
@@ -310,6 +316,42 @@ double oracle_swiglu(double gate, double up, double alpha, double limit, int def
     return (u + 1.0) * g / (1.0 + exp(-alpha * g));
 }
 
+/* ---- planted mistake 12 (model of a dropped second split term) --------------- */
+/* Round to the nearest E4M3 value [F8], ties to even: 3 fraction bits in the normal
+ * range (|r| >= 2^-6), the fixed subnormal spacing 2^-9 below it; magnitudes stay far
+ * below 448 here, so there is no saturation. */
+static double e4m3_round(double r)
+{
+    double a = fabs(r);
+    if (a == 0.0)
+        return r;
+    int e2;
+    frexp(a, &e2);              /* a in [2^(e2-1), 2^e2) */
+    int e = e2 - 1;
+    if (e < -6)
+        e = -6;
+    double q = ldexp(1.0, e - 3);
+    return copysign(nearbyint(a / q) * q, r);
+}
+
+/* v[0..n) in blocks of 32: each block scaled by 2^(e-7), e = floor(log2 of its
+ * largest magnitude), rounded to E4M3 and scaled back. */
+static void keep_e4m3_hi_term(double *v, int64_t n)
+{
+    for (int64_t b0 = 0; b0 < n; b0 += 32) {
+        double amax = 0.0;
+        for (int64_t i = b0; i < b0 + 32 && i < n; ++i)
+            amax = fmax(amax, fabs(v[i]));
+        if (amax == 0.0)
+            continue;
+        int e2;
+        frexp(amax, &e2);
+        double S = ldexp(1.0, (e2 - 1) - 7);
+        for (int64_t i = b0; i < b0 + 32 && i < n; ++i)
+            v[i] = e4m3_round(v[i] / S) * S;
+    }
+}
+
 /* ---- formulation A: per-token loop, weights decoded on the fly -------------- */
 /* For each listed token t (token_list[r], r < n_list):
  *   weight on output (flags = 0):
@@ -363,6 +405,8 @@ static void forward_tokens_impl(int fmt, const uint16_t *x, int64_t T, int64_t H
             int woi = (flags & ORACLE_FLAG_WEIGHT_ON_INPUT) != 0;
             for (int64_t c = 0; c < H; ++c)
                 xin[c] = oracle_bf16_to_double(x[t * H + c]) * (woi ? wj : 1.0);
+            if (defect == ORACLE_DEFECT_OPERAND_E4M3_HI_ONLY)
+                keep_e4m3_hi_term(xin, H);
             /* gate_up projection with bias before the activation [P3] */
             for (int64_t n = 0; n < N_gu; ++n) {
                 double acc = 0.0;
@@ -393,6 +437,8 @@ static void forward_tokens_impl(int fmt, const uint16_t *x, int64_t T, int64_t H
                 }
                 a[i] = oracle_swiglu(gate, up, alpha, limit, defect);
             }
+            if (defect == ORACLE_DEFECT_OPERAND_E4M3_HI_ONLY)
+                keep_e4m3_hi_term(a, I);
             /* down projection; bias added before the routing weight [P3] */
             for (int64_t c = 0; c < H; ++c) {
                 double acc = 0.0, mag = 0.0;

@@ -90,6 +90,19 @@ def test_full_size_workloads_every_tile(moe_gpu, oracle_mod, name):
     _check_layer(moe_gpu, oracle_mod, workload(name), stratified=True)
 
 
+@pytest.mark.parametrize("name", ["tiny_wide", "20b_decode_wide_T8"])
+def test_decode_split_worst_case(moe_gpu, oracle_mod, name):
+    # decode tiles split each bf16 activation into two E4M3 terms per 32-element block;
+    # elements below about 2^-14 of their block's largest one keep only part of their
+    # residual.  Blocks spanning 2^20 and heavy gate biases (activations near zero
+    # beside large ones) put many elements there; the layer must still meet the
+    # configured tolerance (a kernel that dropped the second term would miss it by far:
+    # tests/test_oracle_pins.py::test_dropped_second_split_term_exceeds_layer_tolerance)
+    layer = workload(name)
+    assert moe_gpu.moe_token_tile_rows(layer.T, layer.H, layer.I, layer.E, layer.k) == 32
+    _check_layer(moe_gpu, oracle_mod, layer)
+
+
 def test_route_then_forward_end_to_end(moe_gpu, oracle_mod):
     import torch
     layer = workload("20b_decode_T64")

@@ -419,3 +419,19 @@ def test_envelope_bounds_output_and_matches_dense_special_case(oracle_mod, tiny_
     act = np.vectorize(oracle_mod.swiglu)(h[:, 0::2], h[:, 1::2])
     want = np.abs(act) @ np.abs(Wd.astype(np.float64)).T + np.abs(layer.down_bias[0].astype(np.float64))
     assert rel_l2(env, want) < 1e-12
+
+
+@pytest.mark.parametrize("layer_name", ["tiny_wide", "20b_decode_wide_T8"])
+def test_dropped_second_split_term_exceeds_layer_tolerance(oracle_mod, layer_name):
+    # The decode tiles feed the tensor core two E4M3 terms per activation element at a
+    # power-of-two scale per 32-element block; on blocks spanning 2^20 a kernel that
+    # kept only the first term would be off by far more than the layer tolerance, so
+    # the GPU test on these layers (tests/test_gpu_forward.py) fails if it does.
+    layer = workload(layer_name)
+    ids, w = oracle_mod.route(layer.logits, layer.k)
+    args = (layer.x_bits, ids, w, layer.gate_up.blocks, layer.gate_up.scales, layer.gate_up_bias,
+            layer.down.blocks, layer.down.scales, layer.down_bias)
+    want = oracle_mod.forward_tokens(*args)
+    bad = oracle_mod.forward_tokens(*args, defect=oracle_mod.DEFECT_OPERAND_E4M3_HI_ONLY)
+    assert rel_l2(bad, want) > 2 * REL_L2_TOL
+    assert max_abs_over_rms(bad, want) > 2 * MAX_ABS_OVER_RMS_TOL
