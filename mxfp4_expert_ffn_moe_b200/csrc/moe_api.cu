@@ -12,11 +12,14 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
+#include <stdlib.h>
 
 #include "../../include/moe_mxfp4.h"
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
+#include "gemm_dec.cuh"
 #include "gemm_mxf.cuh"
 #include "gemm_swap.cuh"
 #include "permute.cuh"
@@ -72,6 +75,29 @@ bool forward_sizes_ok(int64_t T, int64_t H, int64_t I, int64_t E, int k) {
 }
 
 int launch_check() { return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// An NVTX range around one entry point (named on a profiler's timeline; free when no
+// tool is attached).
+class NvtxRange {
+   public:
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
+// Average (token, slot) pairs per expert up to which the layer uses decode tiles:
+// MOE_DECODE_MAX_TOKENS_PER_EXPERT from the environment (read once; a non-negative
+// integer), 32 by default (FreeToken PR #838's mmvq_max_tokens plays the same role
+// between its decode and prefill kernels).
+int64_t decode_max_tokens_per_expert() {
+    static const int64_t v = [] {
+        const char *e = getenv("MOE_DECODE_MAX_TOKENS_PER_EXPERT");
+        if (!e || !*e) return (int64_t)32;
+        char *end = nullptr;
+        const long long x = strtoll(e, &end, 10);
+        return (end && *end == '\0' && x >= 0 && x <= (1ll << 30)) ? (int64_t)x : (int64_t)32;
+    }();
+    return v;
+}
 
 // Launch with programmatic stream serialisation: the kernel may be scheduled while
 // its predecessor in the stream is still running; every kernel of the layer calls
@@ -216,6 +242,36 @@ bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int6
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// packed MXFP4 codes [E, N, K/2] as 4-bit elements that the TMA writes "unpacked"
+// (16 codes in the first 8 bytes of each 16-byte chunk), 128-byte swizzle: box of 128
+// elements x 128 rows x 1 expert over the first K_full = 128 * floor(K / 128) elements
+// of each row.  Needs a 32-byte aligned base and K >= 128.
+bool make_unpack_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc || K < 128 || !aligned(ptr, 32) || (K / 2) % 32 != 0) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 128 * 128), (cuuint64_t)N, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
+    cuuint32_t box[3] = {128u, (cuuint32_t)moe::dec::BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// the packed bytes of each row's last 64 elements when K is not a multiple of 128:
+// box of 32 bytes x 128 rows x 1 expert (no swizzle)
+bool make_tail_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
+    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
+    cuuint32_t box[3] = {moe::dec::TAIL_ROW, (cuuint32_t)moe::dec::BM, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int max_smem_optin() {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -328,6 +384,54 @@ int launch_mxf_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const ui
     return launch_check();
 }
 
+// Block-scaled grouped projection for decode tiles (gemm_dec.cuh): split rows B
+// ([2][P][K] + scale slots) x packed weights [E, N, K/2] of each row's expert.
+template <bool kGateUp>
+int launch_dec_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const uint8_t *wblocks,
+                    const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
+                    const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
+                    uint8_t *actq, float alpha, float limit, float *yp,
+                    const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
+    CUtensorMap ma, mt, mb, mbs;
+    if (!make_unpack_map(&ma, wblocks, E, N, K) || !make_split_map(&mb, bq, P, K) ||
+        !make_split_scale_map(&mbs, bq, P, K))
+        return MOE_ERR_CUDA;
+    if (K % 128 != 0) {
+        if (!make_tail_map(&mt, wblocks, E, N, K)) return MOE_ERR_CUDA;
+    } else {
+        mt = ma;   // no tail steps: never read
+    }
+    moe::dec::Params p{};
+    p.counts = counts;
+    p.offsets = offsets;
+    p.tile_offsets = tile_offsets;
+    p.wscales = wscales;
+    p.bias = bias;
+    p.E = (int)E;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.P = (int)P;
+    p.K_full = (int)(K / 128 * 128);
+    p.actq = actq;
+    p.alpha = alpha;
+    p.limit = limit;
+    p.yp = yp;
+    p.sorted_pairs = sorted_pairs;
+    p.weights = weights;
+    p.weight_on_input = woi;
+    const uint32_t smem = moe::dec::smem_bytes((int)(K / 32));
+    if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
+    auto kernel = moe::dec::grouped_mxfp4_dec_kernel<kGateUp>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const int64_t w_tiles = moe::ceil_div(N, moe::dec::BM);
+    const int64_t max_items = (moe::ceil_div(P, moe::dec::TOK) + E) * w_tiles;
+    const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
+    StageScope scope(stage, s);
+    launch_pdl(kernel, dim3(grid), dim3(moe::dec::kThreads), smem, s, ma, mt, mb, mbs, p);
+    return launch_check();
+}
+
 // Split of the gathered rows, then both projections on the block-scaled path.
 template <class Cfg>
 int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sorted_pairs,
@@ -346,6 +450,7 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
     }
     int rc = launch_check();
     if (rc != MOE_OK) return rc;
+#if MOE_DEC_LEGACY
     rc = launch_mxf_gemm<Cfg, true>(MOE_STAGE_GATE_UP, xq, P, H, gate_up_blocks, gate_up_scales,
                                     gate_up_bias, E, 2 * I, counts, offsets, tile_offsets, actq,
                                     alpha, limit, nullptr, sorted_pairs, weights, 0, s);
@@ -353,11 +458,20 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
     return launch_mxf_gemm<Cfg, false>(MOE_STAGE_DOWN, actq, P, I, down_blocks, down_scales,
                                        down_bias, E, H, counts, offsets, tile_offsets, nullptr,
                                        alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
+#else
+    rc = launch_dec_gemm<true>(MOE_STAGE_GATE_UP, xq, P, H, gate_up_blocks, gate_up_scales, gate_up_bias, E,
+                               2 * I, counts, offsets, tile_offsets, actq, alpha, limit, nullptr, sorted_pairs,
+                               weights, 0, s);
+    if (rc != MOE_OK) return rc;
+    return launch_dec_gemm<false>(MOE_STAGE_DOWN, actq, P, I, down_blocks, down_scales, down_bias, E, H, counts,
+                                  offsets, tile_offsets, nullptr, alpha, limit, yp, sorted_pairs, weights,
+                                  woi ? 1 : 0, s);
+#endif
 }
 
 // Token tiles of 32 rows (deep weight pipeline) when experts see few rows on
-// average, 256-row tiles otherwise.
-bool use_decode_tiles(int64_t P, int64_t E) { return P <= 32 * E; }
+// average (decode_max_tokens_per_expert), 256-row tiles otherwise.
+bool use_decode_tiles(int64_t P, int64_t E) { return P <= decode_max_tokens_per_expert() * E; }
 
 // Tile configurations of the grouped GEMMs: the block-scaled kernel (decode tiles) holds
 // two tiles' scale rows (128 x K/32 bytes each) in shared memory; for K too large for
@@ -366,6 +480,9 @@ enum TileConfig { kDecodeSmem, kPrefillSmem, kDecodeMxf, kPrefillMxf };
 
 #ifndef MOE_MXF_DECODE
 #define MOE_MXF_DECODE 1
+#endif
+#ifndef MOE_DEC_LEGACY
+#define MOE_DEC_LEGACY 0
 #endif
 #ifndef MOE_MXF_PREFILL
 #define MOE_MXF_PREFILL 0
@@ -379,10 +496,17 @@ bool config_fits(int64_t H, int64_t I) {
 
 // NVFP4 banks always take the converter kernel: the block-scaled MMA of the decode
 // tiles reads E8M0 scales per 32 elements only.
+bool dec_fits(int64_t H, int64_t I) {
+    if (MOE_DEC_LEGACY) return config_fits<moe::mxf::DecodeCfg>(H, I);
+    const int optin = max_smem_optin();
+    return H >= 128 && I >= 128 && (int)moe::dec::smem_bytes((int)(H / 32)) <= optin &&
+           (int)moe::dec::smem_bytes((int)(I / 32)) <= optin;
+}
+
 TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E, bool nv) {
     if (nv) return use_decode_tiles(P, E) ? kDecodeSmem : kPrefillSmem;
     if (use_decode_tiles(P, E))
-        return (MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) ? kDecodeMxf : kDecodeSmem;
+        return (MOE_MXF_DECODE && dec_fits(H, I)) ? kDecodeMxf : kDecodeSmem;
     return (MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) ? kPrefillMxf : kPrefillSmem;
 }
 
@@ -463,7 +587,10 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     float *yp = rows_out ? rows_out : reinterpret_cast<float *>(ws + L.yp);
 
     const int64_t P = T * k;
-    const TileConfig cfg = pick_config(P, H, I, E, nv);
+    TileConfig cfg = pick_config(P, H, I, E, nv);
+    // the decode kernel's weight loads unpack 4-bit codes, which needs 32-byte aligned banks
+    if (cfg == kDecodeMxf && !MOE_DEC_LEGACY && (!aligned(gate_up_blocks, 32) || !aligned(down_blocks, 32)))
+        cfg = kDecodeSmem;
     int rc = MOE_OK;
     do {
         if ((rc = launch_permute(ids, (int)expert_base, P, E, config_tok(cfg), counts, offsets, tile_offsets,
@@ -607,16 +734,19 @@ const char *moe_status_string(int status) {
 
 int mxfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, uint16_t *out, int64_t E,
                      int64_t N, int64_t K, void *stream) {
+    NvtxRange nvtx("mxfp4_dequantize");
     return launch_mxfp4_dequant<false>(blocks, scales, out, E, N, K, (cudaStream_t)stream);
 }
 
 int nvfp4_dequantize(const uint8_t *blocks, const uint8_t *scales, const float *scale2, uint16_t *out,
                      int64_t E, int64_t N, int64_t K, void *stream) {
+    NvtxRange nvtx("nvfp4_dequantize");
     return launch_nvfp4_dequant<false>(blocks, scales, scale2, out, E, N, K, (cudaStream_t)stream);
 }
 
 int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales, uint16_t *out,
                                int64_t E, int64_t N, int64_t K, void *stream) {
+    NvtxRange nvtx("mxfp4_dequantize_from_host");
     if (!host_blocks || !host_scales || !out || !bank_sizes_ok(E, N, K, 32)) return MOE_ERR_INVALID_ARG;
     const void *db = nullptr, *ds = nullptr;
     int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
@@ -629,6 +759,7 @@ int mxfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_s
 int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_scales,
                                const float *scale2, uint16_t *out, int64_t E, int64_t N, int64_t K,
                                void *stream) {
+    NvtxRange nvtx("nvfp4_dequantize_from_host");
     if (!host_blocks || !host_scales || !out || !bank_sizes_ok(E, N, K, 16)) return MOE_ERR_INVALID_ARG;
     const void *db = nullptr, *ds = nullptr;
     int rc = device_view_of_host(host_blocks, E * N * (K / 2), &db);
@@ -640,6 +771,7 @@ int nvfp4_dequantize_from_host(const uint8_t *host_blocks, const uint8_t *host_s
 
 int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *ids,
               float *weights, void *stream) {
+    NvtxRange nvtx("moe_route");
     if (!router_logits || !ids || !weights) return MOE_ERR_INVALID_ARG;
     if (T < 1 || E < 1 || k < 1 || k > 8 || k > E) return MOE_ERR_INVALID_ARG;
     if (E > 256) return MOE_ERR_UNSUPPORTED;
@@ -669,6 +801,7 @@ int moe_route(const float *router_logits, int64_t T, int64_t E, int k, int32_t *
 int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b_router, int64_t T,
                      int64_t H, int64_t E, int k, float *logits, int32_t *ids, float *weights,
                      void *stream) {
+    NvtxRange nvtx("moe_router_route");
     if (!x || !w_router || !ids || !weights) return MOE_ERR_INVALID_ARG;
     if (T < 1 || T > (int64_t)0x7FFFFFFF - moe::rtr::BM) return MOE_ERR_INVALID_ARG;
     if (H < 64 || H % 64 != 0 || H > (int64_t)0x7FFFFFFF) return MOE_ERR_INVALID_ARG;
@@ -697,6 +830,7 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
 int moe_gather_pairs(const uint16_t *x, int64_t T, int64_t H, int k, const int32_t *ids, const float *weights,
                      const int32_t *sorted_pairs, const int32_t *offsets, int64_t E, uint16_t *x_rows,
                      int32_t *row_ids, float *row_weights, void *stream) {
+    NvtxRange nvtx("moe_gather_pairs");
     if (!x || !ids || !weights || !sorted_pairs || !offsets || !x_rows || !row_ids || !row_weights)
         return MOE_ERR_INVALID_ARG;
     if (T < 1 || k < 1 || k > 8 || E < 1 || E > 256 || H < 8 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
@@ -717,6 +851,7 @@ int moe_mxfp4_expert_rows(const uint16_t *x_rows, int64_t R, int64_t H, int64_t 
                           const uint8_t *down_blocks, const uint8_t *down_scales, const float *down_bias,
                           float alpha, float limit, float *y_rows, uint32_t flags, void *workspace,
                           size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx("moe_mxfp4_expert_rows");
     if (!y_rows) return MOE_ERR_INVALID_ARG;
     return forward_layer(false, x_rows, R, H, I, E, 1, row_ids, row_weights, gate_up_blocks, gate_up_scales,
                          nullptr, gate_up_bias, down_blocks, down_scales, nullptr, down_bias, alpha, limit,
@@ -725,6 +860,7 @@ int moe_mxfp4_expert_rows(const uint16_t *x_rows, int64_t R, int64_t H, int64_t 
 
 int moe_combine_pairs(const float *y_rows, const int32_t *pair_rows, int64_t T, int k, int64_t H, uint16_t *out,
                       void *stream) {
+    NvtxRange nvtx("moe_combine_pairs");
     if (!y_rows || !pair_rows || !out) return MOE_ERR_INVALID_ARG;
     if (T < 1 || k < 1 || k > 8 || H < 4 || H % 4 != 0) return MOE_ERR_INVALID_ARG;
     if (!aligned(y_rows, 16) || !aligned(out, 8)) return MOE_ERR_INVALID_ARG;
@@ -740,6 +876,7 @@ int moe_combine_pairs(const float *y_rows, const int32_t *pair_rows, int64_t T, 
 int moe_permute(const int32_t *ids, int64_t T, int k, int64_t E, int tile_rows, int32_t *counts,
                 int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
                 void *stream) {
+    NvtxRange nvtx("moe_permute");
     if (!ids || !counts || !offsets || !tile_offsets || !sorted_pairs) return MOE_ERR_INVALID_ARG;
     if (T < 1 || k < 1 || k > 8 || E < 1 || E > 256 || tile_rows < 1) return MOE_ERR_INVALID_ARG;
     if (T * k >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -764,6 +901,7 @@ int moe_mxfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                          const uint8_t *down_scales, const float *down_bias, float alpha,
                          float limit, uint16_t *out, uint32_t flags, void *workspace,
                          size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx("moe_mxfp4_forward_ex");
     return forward_layer(false, x, T, H, I, E, k, ids, weights, gate_up_blocks, gate_up_scales, nullptr,
                          gate_up_bias, down_blocks, down_scales, nullptr, down_bias, alpha, limit, out,
                          flags, workspace, workspace_bytes, stream);
@@ -777,6 +915,7 @@ int moe_nvfp4_forward_ex(const uint16_t *x, int64_t T, int64_t H, int64_t I, int
                          const float *down_scale2, const float *down_bias, float alpha,
                          float limit, uint16_t *out, uint32_t flags, void *workspace,
                          size_t workspace_bytes, void *stream) {
+    NvtxRange nvtx("moe_nvfp4_forward_ex");
     return forward_layer(true, x, T, H, I, E, k, ids, weights, gate_up_blocks, gate_up_scales,
                          gate_up_scale2, gate_up_bias, down_blocks, down_scales, down_scale2, down_bias,
                          alpha, limit, out, flags, workspace, workspace_bytes, stream);
@@ -788,6 +927,7 @@ int moe_mxfp4_forward(const uint16_t *x, int64_t T, int64_t H, int64_t I, int64_
                       const uint8_t *down_blocks, const uint8_t *down_scales,
                       const float *down_bias, float alpha, float limit, uint16_t *out,
                       void *stream) {
+    NvtxRange nvtx("moe_mxfp4_forward");
     return moe_mxfp4_forward_ex(x, T, H, I, E, k, ids, weights, gate_up_blocks, gate_up_scales,
                                 gate_up_bias, down_blocks, down_scales, down_bias, alpha, limit,
                                 out, 0u, nullptr, 0, stream);

@@ -139,3 +139,21 @@ def test_nvfp4_router_and_host_copy_argument_checks_need_no_device(lib):
     assert lib.mxfp4_dequantize_from_host(null, p, p, 1, 1, 32, null) == -1
     assert lib.nvfp4_dequantize_from_host(p, p, null, p, 1, 1, 24, null) == -1            # K % 16
     assert lib.nvfp4_dequantize_from_host(p, null, null, p, 1, 1, 16, null) == -1
+
+
+@pytest.mark.parametrize("env,T,want", [(None, 1, 32), (None, 4096, 256), ("0", 1, 256), ("2000", 4096, 32),
+                                        ("junk", 1, 32), ("-5", 4096, 256)])
+def test_decode_switch_environment_override(env, T, want):
+    # MOE_DECODE_MAX_TOKENS_PER_EXPERT moves the decode/prefill tile switch (read once
+    # per process, so each case runs in a fresh interpreter); host-only, no device
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r); import mxfp4_expert_ffn_moe_b200 as m; "
+            "print(m.moe_token_tile_rows(%d, 2880, 2880, 32, 4))" % (ROOT, T))
+    e = dict(os.environ)
+    e.pop("MOE_DECODE_MAX_TOKENS_PER_EXPERT", None)
+    if env is not None:
+        e["MOE_DECODE_MAX_TOKENS_PER_EXPERT"] = env
+    r = subprocess.run([sys.executable, "-c", code], env=e, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr[-400:]
+    assert int(r.stdout.strip().splitlines()[-1]) == want

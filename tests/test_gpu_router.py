@@ -112,3 +112,4 @@ def test_router_nan_logits_follow_the_routing_rule(moe_gpu):
     np.testing.assert_allclose(wt.astype(np.float64).sum(axis=1), 1.0, atol=1e-6)
     ids2, w2 = moe_gpu.moe_route(lg, r.k)
     assert torch.equal(ids2.cpu(), torch.from_numpy(ids)) and torch.equal(w2.cpu(), torch.from_numpy(wt))
+    assert moe_gpu.moe_get_device_error() & moe_gpu.MOE_DEVERR_BAD_LOGIT   # read (and clear) the word
