@@ -5,13 +5,18 @@
 // (golden rel-err 0.0, i.e. exact).  Element kk of a row sits in byte kk/2 (even
 // element in the low nibble) and is scaled by the E8M0 byte kk/32 of that row.
 //
-// HBM-bound streaming kernel.  Each thread turns one 32-bit packed word (eight
-// codes, a quarter of a 32-element scale block) into one 16-byte bf16 chunk, so a
-// warp reads 128 contiguous bytes and writes 512 contiguous bytes per step.  The
-// E2M1 magnitudes come from a 16-entry fp32 table in shared memory (16 distinct
-// banks: no conflicts); values are scaled by an exact fp32 power of two and
-// rounded to bf16, which never rounds for scale bytes <= 252 and gives the bf16
-// subnormals / infinities of the exact product for the extreme bytes.
+// HBM-bound streaming kernel with a write-heavy mix (4.25 bits read per 16 written).
+// Each thread decodes one 32-bit packed word (eight codes, a quarter of a 32-element
+// scale block) with integer operations and packed bf16 multiplies, no table: the
+// codes become the bf16 bit patterns of E2M1 * 2^-126 (sign to bit 15, exponent bits
+// and mantissa msb to bits 8..6; code 1 = 0.5 is the subnormal 2^-127), then one bf16
+// multiply by 2^(s-1) (two, by 2^126 and 2^(s-127), when s > 128) gives
+// E2M1 * 2^(s-127), rounded to nearest even only where that is a bf16 subnormal or
+// overflows -- the exact product otherwise.  A block of 256 threads decodes 1024
+// consecutive words into 16 KB of shared memory and one bulk asynchronous copy writes
+// it out (double-buffered); reads are coalesced 4-byte loads.  Measured on the
+// gpt-oss-20b bank: bulk stores of 16 KB runs beat direct 16-byte stores by ~7 %, and
+// one 16-byte load plus four strided 16-byte stores per thread lose ~30 %.
 //
 // Both decode kernels also serve dequant-on-copy from host memory (kHostSrc): the
 // packed bank stays in page-locked host memory, the kernel reads it through its
@@ -46,63 +51,90 @@ __device__ __forceinline__ uint32_t load_byte(const uint8_t *p) {
     }
 }
 
-template <bool kHostSrc>
-__global__ void __launch_bounds__(256) mxfp4_dequant_kernel(const uint32_t *__restrict__ packed,
-                                                            const uint8_t *__restrict__ scales,
-                                                            uint4 *__restrict__ out,
-                                                            int64_t n_words) {
-    __shared__ float lut[16];
-    if (threadIdx.x < 16) {
-        // E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0.
-        const uint32_t c = threadIdx.x, e = (c >> 1) & 3u, m = c & 1u;
-        float mag = (e == 0u) ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, (int)e - 1);
-        lut[c] = (c & 8u) ? -mag : mag;
+// Eight E2M1 codes (element 2j in the low nibble of byte j) -> four bf16x2 words of
+// E2M1 * 2^(s - 127) for the multipliers of scale_multipliers.
+__device__ __forceinline__ uint4 e2m1x8_scaled(uint32_t q, uint32_t m1, uint32_t m2) {
+    const uint32_t lo = q & 0x0F0F0F0Fu, hi = (q >> 4) & 0x0F0F0F0Fu;
+    uint32_t r[4];
+    asm("prmt.b32 %0, %1, %2, 0x8480;" : "=r"(r[0]) : "r"(lo), "r"(hi));
+    asm("prmt.b32 %0, %1, %2, 0x8581;" : "=r"(r[1]) : "r"(lo), "r"(hi));
+    asm("prmt.b32 %0, %1, %2, 0x8682;" : "=r"(r[2]) : "r"(lo), "r"(hi));
+    asm("prmt.b32 %0, %1, %2, 0x8783;" : "=r"(r[3]) : "r"(lo), "r"(hi));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        r[i] = (r[i] * 0x1040u) & 0x81C081C0u;   // sign, exponent bits, mantissa msb
+        asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r[i]) : "r"(r[i]), "r"(m1));
+        if (m2) asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r[i]) : "r"(r[i]), "r"(m2));
     }
-    __syncthreads();
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
 
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    constexpr int U = 4;
-    for (; w + (U - 1) * stride < n_words; w += U * stride) {
-        uint32_t word[U], s[U];
+// bf16x2 multipliers taking E2M1 * 2^-126 to E2M1 * 2^(s - 127): one (2^(s - 1)) when
+// that is a normal bf16, else 2^126 then 2^(s - 127).
+__device__ __forceinline__ void scale_multipliers(uint32_t s, uint32_t &m1, uint32_t &m2) {
+    if (s <= 128u) {
+        m1 = ((s + 126u) << 7) * 0x10001u;
+        m2 = 0u;
+    } else {
+        m1 = 0x7E807E80u;
+        m2 = (s << 7) * 0x10001u;
+    }
+}
+
+template <bool kHostSrc>
+__device__ __forceinline__ uint4 dequant_word(uint32_t q, uint32_t s) {
+    if (s == 255u) {   // invalid scale byte: NaN and the device error word
+        raise_device_error(MOE_DEVERR_BAD_SCALE);
+        return make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+    }
+    uint32_t m1, m2;
+    scale_multipliers(s, m1, m2);
+    return e2m1x8_scaled(q, m1, m2);
+}
+
+constexpr int kDequantThreads = 256;
+constexpr int kDequantWords = 4 * kDequantThreads;   // words per round (16 KB of bf16)
+
+// Block b decodes words [b * words_per_block, (b + 1) * words_per_block) of the bank
+// (words_per_block a multiple of kDequantWords); each round's 16 KB leaves with one
+// bulk copy from shared memory.
+template <bool kHostSrc>
+__global__ void __launch_bounds__(kDequantThreads) mxfp4_dequant_kernel(const uint32_t *__restrict__ packed,
+                                                                        const uint8_t *__restrict__ scales,
+                                                                        uint4 *__restrict__ out, int64_t n_words,
+                                                                        int64_t words_per_block) {
+    __shared__ __align__(128) uint4 stage[2][kDequantWords];
+    const int64_t w0 = (int64_t)blockIdx.x * words_per_block;
+    const int64_t w1 = min(n_words, w0 + words_per_block);
+    int round = 0;
+    for (int64_t base = w0; base < w1; base += kDequantWords, ++round) {
+        const int b = round & 1;
+        if (round >= 2) {
+            // the copy that read this buffer two rounds ago has finished reading it
+            if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            __syncthreads();
+        }
+        const int64_t n = min((int64_t)kDequantWords, w1 - base);
+        uint32_t q[4], sb[4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            word[u] = load_word<kHostSrc>(packed + w + u * stride);
-            s[u] = load_byte<kHostSrc>(scales + ((w + u * stride) >> 2));  // 4 words per 32-element block
+        for (int u = 0; u < 4; ++u) {
+            const int64_t i = base + threadIdx.x + kDequantThreads * u;
+            q[u] = i < w1 ? load_word<kHostSrc>(packed + i) : 0u;
+            sb[u] = i < w1 ? load_byte<kHostSrc>(scales + (i >> 2)) : 127u;   // 4 words per scale block
         }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            uint4 v;
-            if (s[u] == 255u) {
-                raise_device_error(MOE_DEVERR_BAD_SCALE);
-                v = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
-            } else {
-                const float sc = e8m0_to_f32(s[u]);
-                const uint32_t q = word[u];
-                v.x = pack_bf16x2(lut[q & 15u] * sc, lut[(q >> 4) & 15u] * sc);
-                v.y = pack_bf16x2(lut[(q >> 8) & 15u] * sc, lut[(q >> 12) & 15u] * sc);
-                v.z = pack_bf16x2(lut[(q >> 16) & 15u] * sc, lut[(q >> 20) & 15u] * sc);
-                v.w = pack_bf16x2(lut[(q >> 24) & 15u] * sc, lut[q >> 28] * sc);
-            }
-            __stcs(out + w + u * stride, v);
+        for (int u = 0; u < 4; ++u) stage[b][threadIdx.x + kDequantThreads * u] = dequant_word<kHostSrc>(q[u], sb[u]);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(out + base),
+                         "r"((uint32_t)__cvta_generic_to_shared(&stage[b][0])), "r"((uint32_t)(n * 16))
+                         : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
     }
-    for (; w < n_words; w += stride) {
-        const uint32_t q = load_word<kHostSrc>(packed + w);
-        const uint32_t sb = load_byte<kHostSrc>(scales + (w >> 2));
-        uint4 v;
-        if (sb == 255u) {
-            raise_device_error(MOE_DEVERR_BAD_SCALE);
-            v = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
-        } else {
-            const float sc = e8m0_to_f32(sb);
-            v.x = pack_bf16x2(lut[q & 15u] * sc, lut[(q >> 4) & 15u] * sc);
-            v.y = pack_bf16x2(lut[(q >> 8) & 15u] * sc, lut[(q >> 12) & 15u] * sc);
-            v.z = pack_bf16x2(lut[(q >> 16) & 15u] * sc, lut[(q >> 20) & 15u] * sc);
-            v.w = pack_bf16x2(lut[(q >> 24) & 15u] * sc, lut[q >> 28] * sc);
-        }
-        __stcs(out + w, v);
-    }
+    // the copies must have read shared memory before the block exits
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---- NVFP4 ------------------------------------------------------------------

@@ -102,7 +102,10 @@ struct Config {
     static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES;
     static constexpr uint32_t OFF_XCH = OFF_EPI + kEpiStage * kEpiWarps;
     static constexpr uint32_t OFF_SINK = OFF_XCH + kXchBytes;
-    static constexpr uint32_t OFF_BAR = OFF_SINK + kSinkBytes;
+    // the tile schedule (counts, row offsets, tile offsets; E <= 256) staged per CTA
+    static constexpr uint32_t OFF_SCHED = OFF_SINK + kSinkBytes;
+    static constexpr uint32_t OFF_BAR = (OFF_SCHED + 3 * 4 * 257 + 15u) & ~15u;   // mbarriers: 8-byte aligned
+    static_assert(OFF_BAR % 16 == 0, "barrier alignment");
     static constexpr uint32_t BAR_BYTES = 8 * (3 * S + 2 * PS + 2 * NACC + 6) + 16;
     static constexpr uint32_t OFF_SC = (OFF_BAR + BAR_BYTES + 127u) & ~127u;
     static constexpr uint32_t SMEM_FIXED = OFF_SC + 1024;   // + slack for the 1 KB base alignment
@@ -145,11 +148,17 @@ struct Params {
     int weight_on_input;
 };
 
-__device__ __forceinline__ int tile_expert(const int32_t *__restrict__ tile_offsets, int E, int m) {
+// The schedule a CTA stages in shared memory once, so that each role decodes its
+// work items without dependent global loads.
+struct Sched {
+    const int *counts, *offsets, *tile_offsets;
+};
+
+__device__ __forceinline__ int tile_expert(const int *tile_offsets, int E, int m) {
     int lo = 0, hi = E - 1;  // largest e with tile_offsets[e] <= m
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(tile_offsets + mid) <= m)
+        if (tile_offsets[mid] <= m)
             lo = mid;
         else
             hi = mid - 1;
@@ -169,14 +178,14 @@ struct Tile {
 // Work item -> tile; the weight tile index runs fastest, so the CTAs running at one
 // time share token tiles through L2.
 template <int TOK>
-__device__ __forceinline__ Tile decode_tile(const Params &p, int item, int w_tiles) {
+__device__ __forceinline__ Tile decode_tile(const Params &p, const Sched &sc, int item, int w_tiles) {
     Tile t;
     const int g = item / w_tiles;
     const int wt = item - g * w_tiles;
-    t.e = tile_expert(p.tile_offsets, p.E, g);
-    const int tt = g - __ldg(p.tile_offsets + t.e);
-    t.row0 = __ldg(p.offsets + t.e) + tt * TOK;
-    t.ntok = min(TOK, __ldg(p.counts + t.e) - tt * TOK);
+    t.e = tile_expert(sc.tile_offsets, p.E, g);
+    const int tt = g - sc.tile_offsets[t.e];
+    t.row0 = sc.offsets[t.e] + tt * TOK;
+    t.ntok = min(TOK, sc.counts[t.e] - tt * TOK);
     t.h = (t.ntok + 15) & ~15;
     t.m0 = wt * BM;
     t.mrows = min(BM, p.N - t.m0);
@@ -271,13 +280,22 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // barriers and TMEM are set up; wait for the producer of this kernel's inputs
+    // barriers and TMEM are set up; wait for the producer of this kernel's inputs, then
+    // stage the schedule it wrote
     pdl_wait();
     pdl_trigger();
+    int *const s_sched = reinterpret_cast<int *>(gbase + Cfg::OFF_SCHED);
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+        s_sched[i] = i < p.E ? __ldg(p.counts + i) : 0;
+        s_sched[257 + i] = __ldg(p.offsets + i);
+        s_sched[514 + i] = __ldg(p.tile_offsets + i);
+    }
+    __syncthreads();
+    const Sched sc{s_sched, s_sched + 257, s_sched + 514};
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gbase + (tmem_holder - base));
 
     const int w_tiles = (p.N + BM - 1) / BM;
-    const int total = __ldg(p.tile_offsets + p.E) * w_tiles;
+    const int total = sc.tile_offsets[p.E] * w_tiles;
     // K steps per tile, rounded up to KALIGN: the extra steps read only the TMA's zero
     // fill (codes and token rows past K) with scale 1 and add nothing
     const int k_iters = ((p.K + BK - 1) / BK + Cfg::KALIGN - 1) / Cfg::KALIGN * Cfg::KALIGN;
@@ -288,7 +306,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, sc, item, w_tiles);
             const int nbox = t.h / XBOX_ROWS;
             for (int kb = 0; kb < k_iters; ++kb, ++it) {
                 const int s = it % S;
@@ -312,7 +330,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         uint32_t it = 0, local = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, sc, item, w_tiles);
             const int sb = local & 1;
             if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(sc_empty(sb), ((local >> 1) & 1u) ^ 1u)))) break;
             if (ptx::elect_one()) {
@@ -337,7 +355,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         uint32_t it = 0, local = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, sc, item, w_tiles);
             const uint32_t idesc = idesc_e2m1_e4m3(BM, 2 * t.h);
             const int b = local % NACC;
             if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_empty(b), ((local / NACC) & 1u) ^ 1u)))) break;
@@ -374,7 +392,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         uint32_t local = 0, chunk = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, sc, item, w_tiles);
             const int b = local % NACC;
             if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_full(b), (local / NACC) & 1u))) break;
             ptx::tc_fence_after();
@@ -458,9 +476,23 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
                         *reinterpret_cast<uint4 *>(lrow + f0) = make_uint4(lq[0], lq[1], lq[2], lq[3]);
                         if ((q & 1) == 0) {   // one warp of the pair writes the block's scale bytes
                             const int blk = f0 >> 5;
-                            const int64_t at = I + 16 * (blk >> 2) + (blk & 3);
-                            hrow[at] = (uint8_t)bsc;
-                            lrow[at] = (uint8_t)(bsc - 4u);
+                            const int64_t slot = I + 16 * (blk >> 2);
+                            hrow[slot + (blk & 3)] = (uint8_t)bsc;
+                            lrow[slot + (blk & 3)] = (uint8_t)(bsc - 4u);
+                            if ((blk & 3) == 0) {
+                                // the writer of a step's first block completes the slot the
+                                // way the token split does: scale 1 (127) for blocks past I,
+                                // zeros after the scale word, so no byte of the slot is left
+                                // from an earlier call
+                                const int nblk = I / 32;
+#pragma unroll
+                                for (int j = 1; j < 4; ++j)
+                                    if (blk + j >= nblk) hrow[slot + j] = lrow[slot + j] = 127u;
+                                uint32_t *hw = reinterpret_cast<uint32_t *>(hrow + slot);
+                                uint32_t *lw = reinterpret_cast<uint32_t *>(lrow + slot);
+                                hw[1] = hw[2] = hw[3] = 0u;
+                                lw[1] = lw[2] = lw[3] = 0u;
+                            }
                         }
                     }
                     __syncwarp();
@@ -519,7 +551,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
         uint32_t it = 0, local = 0, pit = 0;   // step and packed-load counters of this CTA
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local, pit += wp_loads) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, sc, item, w_tiles);
             const int sb = local & 1;
             // every stager warp takes part in every tile's scale slot (even with no step
             // of its own in the tile), so that the slot's arrival count never mixes tiles

@@ -90,7 +90,10 @@ struct Config {
     static constexpr uint32_t OFF_X = OFF_WB + S * WB_BYTES;    // S x tokens
     static constexpr uint32_t OFF_WP = OFF_X + S * X_BYTES;     // PS x 4 KB packed weights
     static constexpr uint32_t OFF_EPI = OFF_WP + PS * WP_BYTES; // epilogue staging, 4 KB / warp
-    static constexpr uint32_t OFF_BAR = OFF_EPI + 4096 * kEpiWarps;
+    // the tile offsets (E <= 256) staged per CTA for the item -> expert search
+    static constexpr uint32_t OFF_TOFF = OFF_EPI + 4096 * kEpiWarps;
+    static constexpr uint32_t OFF_BAR = (OFF_TOFF + 4 * 257 + 15u) & ~15u;   // mbarriers: 8-byte aligned
+    static_assert(OFF_BAR % 16 == 0, "barrier alignment");
     static constexpr uint32_t BAR_BYTES = 8 * (2 * S + 2 * PS + 2 * NACC) + 16;
     // + slack for aligning the base to 1 KB
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024;
@@ -124,11 +127,12 @@ struct Params {
     int weight_on_input;
 };
 
-__device__ __forceinline__ int tile_expert(const int32_t *__restrict__ tile_offsets, int E, int m) {
+// s_toff: the tile offsets staged in shared memory
+__device__ __forceinline__ int tile_expert(const int *s_toff, int E, int m) {
     int lo = 0, hi = E - 1;  // largest e with tile_offsets[e] <= m
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(tile_offsets + mid) <= m)
+        if (s_toff[mid] <= m)
             lo = mid;
         else
             hi = mid - 1;
@@ -147,12 +151,12 @@ struct Tile {
 // Work item -> tile.  Items enumerate (token tile, weight tile) with the weight
 // tile fastest, so the CTAs running at one time share token tiles through L2.
 template <int TOK>
-__device__ __forceinline__ Tile decode_tile(const Params &p, int item, int w_tiles) {
+__device__ __forceinline__ Tile decode_tile(const Params &p, const int *s_toff, int item, int w_tiles) {
     Tile t;
     const int g = item / w_tiles;
     const int wt = item - g * w_tiles;
-    t.e = tile_expert(p.tile_offsets, p.E, g);
-    const int tt = g - __ldg(p.tile_offsets + t.e);
+    t.e = tile_expert(s_toff, p.E, g);
+    const int tt = g - s_toff[t.e];
     t.row0 = __ldg(p.offsets + t.e) + tt * TOK;
     t.ntok = min(TOK, __ldg(p.counts + t.e) - tt * TOK);
     t.m0 = wt * BM;
@@ -240,13 +244,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // barriers and TMEM are set up; wait for the producer of this kernel's inputs
+    // barriers and TMEM are set up; wait for the producer of this kernel's inputs, then
+    // stage the tile offsets it wrote
     pdl_wait();
     pdl_trigger();
+    int *const s_toff = reinterpret_cast<int *>(gbase + Cfg::OFF_TOFF);
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) s_toff[i] = __ldg(p.tile_offsets + i);
+    __syncthreads();
     const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t *>(gbase + (tmem_holder - base));
 
     const int w_tiles = (p.N + BM - 1) / BM;
-    const int total = __ldg(p.tile_offsets + p.E) * w_tiles;
+    const int total = s_toff[p.E] * w_tiles;
     const int k_iters = p.K / BK;
 
     if (warp == 0) {
@@ -256,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             const int nbox = (t.ntok + (int)XBOX_ROWS - 1) / (int)XBOX_ROWS;
             for (int kb = 0; kb < k_iters; ++kb, ++it) {
                 const int s = it % S;
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             for (int kb = 0; kb < k_iters; ++kb, ++it) {
                 const int s = it % PS;
                 if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_empty(s), ((it / PS) & 1u) ^ 1u)))) break;
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0, local = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             const int nmma = max(16, (t.ntok + 15) & ~15);
             const uint32_t idesc = ptx::idesc_bf16_f32(BM, nmma);
             const int b = local % Cfg::NACC;
@@ -323,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = q * 32 + lane;             // weight row within the tile
         uint32_t local = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++local) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             const int b = local % Cfg::NACC;
             if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_full(b), (local / Cfg::NACC) & 1u))) break;
             ptx::tc_fence_after();
@@ -451,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Tile t = decode_tile<TOK>(p, item, w_tiles);
+            const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             const uint8_t *srow[kBlocksPerThread];
             bool rok[kBlocksPerThread];
 #pragma unroll

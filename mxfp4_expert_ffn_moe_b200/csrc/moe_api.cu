@@ -19,7 +19,6 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
-#include "gemm_dec.cuh"
 #include "gemm_mxf.cuh"
 #include "gemm_swap.cuh"
 #include "permute.cuh"
@@ -242,36 +241,6 @@ bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int6
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// packed MXFP4 codes [E, N, K/2] as 4-bit elements that the TMA writes "unpacked"
-// (16 codes in the first 8 bytes of each 16-byte chunk), 128-byte swizzle: box of 128
-// elements x 128 rows x 1 expert over the first K_full = 128 * floor(K / 128) elements
-// of each row.  Needs a 32-byte aligned base and K >= 128.
-bool make_unpack_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
-    auto enc = tensor_map_encoder();
-    if (!enc || K < 128 || !aligned(ptr, 32) || (K / 2) % 32 != 0) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)(K / 128 * 128), (cuuint64_t)N, (cuuint64_t)E};
-    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
-    cuuint32_t box[3] = {128u, (cuuint32_t)moe::dec::BM, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// the packed bytes of each row's last 64 elements when K is not a multiple of 128:
-// box of 32 bytes x 128 rows x 1 expert (no swizzle)
-bool make_tail_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int64_t K) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)(K / 2), (cuuint64_t)N, (cuuint64_t)E};
-    cuuint64_t strides[2] = {(cuuint64_t)(K / 2), (cuuint64_t)(N * (K / 2))};
-    cuuint32_t box[3] = {moe::dec::TAIL_ROW, (cuuint32_t)moe::dec::BM, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int max_smem_optin() {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -384,54 +353,6 @@ int launch_mxf_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const ui
     return launch_check();
 }
 
-// Block-scaled grouped projection for decode tiles (gemm_dec.cuh): split rows B
-// ([2][P][K] + scale slots) x packed weights [E, N, K/2] of each row's expert.
-template <bool kGateUp>
-int launch_dec_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const uint8_t *wblocks,
-                    const uint8_t *wscales, const float *bias, int64_t E, int64_t N,
-                    const int32_t *counts, const int32_t *offsets, const int32_t *tile_offsets,
-                    uint8_t *actq, float alpha, float limit, float *yp,
-                    const int32_t *sorted_pairs, const float *weights, int woi, cudaStream_t s) {
-    CUtensorMap ma, mt, mb, mbs;
-    if (!make_unpack_map(&ma, wblocks, E, N, K) || !make_split_map(&mb, bq, P, K) ||
-        !make_split_scale_map(&mbs, bq, P, K))
-        return MOE_ERR_CUDA;
-    if (K % 128 != 0) {
-        if (!make_tail_map(&mt, wblocks, E, N, K)) return MOE_ERR_CUDA;
-    } else {
-        mt = ma;   // no tail steps: never read
-    }
-    moe::dec::Params p{};
-    p.counts = counts;
-    p.offsets = offsets;
-    p.tile_offsets = tile_offsets;
-    p.wscales = wscales;
-    p.bias = bias;
-    p.E = (int)E;
-    p.N = (int)N;
-    p.K = (int)K;
-    p.P = (int)P;
-    p.K_full = (int)(K / 128 * 128);
-    p.actq = actq;
-    p.alpha = alpha;
-    p.limit = limit;
-    p.yp = yp;
-    p.sorted_pairs = sorted_pairs;
-    p.weights = weights;
-    p.weight_on_input = woi;
-    const uint32_t smem = moe::dec::smem_bytes((int)(K / 32));
-    if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
-    auto kernel = moe::dec::grouped_mxfp4_dec_kernel<kGateUp>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    const int64_t w_tiles = moe::ceil_div(N, moe::dec::BM);
-    const int64_t max_items = (moe::ceil_div(P, moe::dec::TOK) + E) * w_tiles;
-    const int grid = (int)(max_items < sm_count() ? max_items : sm_count());
-    StageScope scope(stage, s);
-    launch_pdl(kernel, dim3(grid), dim3(moe::dec::kThreads), smem, s, ma, mt, mb, mbs, p);
-    return launch_check();
-}
-
 // Split of the gathered rows, then both projections on the block-scaled path.
 template <class Cfg>
 int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sorted_pairs,
@@ -450,7 +371,6 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
     }
     int rc = launch_check();
     if (rc != MOE_OK) return rc;
-#if MOE_DEC_LEGACY
     rc = launch_mxf_gemm<Cfg, true>(MOE_STAGE_GATE_UP, xq, P, H, gate_up_blocks, gate_up_scales,
                                     gate_up_bias, E, 2 * I, counts, offsets, tile_offsets, actq,
                                     alpha, limit, nullptr, sorted_pairs, weights, 0, s);
@@ -458,15 +378,6 @@ int launch_mxf_layer(const uint16_t *x, const float *weights, const int32_t *sor
     return launch_mxf_gemm<Cfg, false>(MOE_STAGE_DOWN, actq, P, I, down_blocks, down_scales,
                                        down_bias, E, H, counts, offsets, tile_offsets, nullptr,
                                        alpha, limit, yp, sorted_pairs, weights, woi ? 1 : 0, s);
-#else
-    rc = launch_dec_gemm<true>(MOE_STAGE_GATE_UP, xq, P, H, gate_up_blocks, gate_up_scales, gate_up_bias, E,
-                               2 * I, counts, offsets, tile_offsets, actq, alpha, limit, nullptr, sorted_pairs,
-                               weights, 0, s);
-    if (rc != MOE_OK) return rc;
-    return launch_dec_gemm<false>(MOE_STAGE_DOWN, actq, P, I, down_blocks, down_scales, down_bias, E, H, counts,
-                                  offsets, tile_offsets, nullptr, alpha, limit, yp, sorted_pairs, weights,
-                                  woi ? 1 : 0, s);
-#endif
 }
 
 // Token tiles of 32 rows (deep weight pipeline) when experts see few rows on
@@ -481,9 +392,7 @@ enum TileConfig { kDecodeSmem, kPrefillSmem, kDecodeMxf, kPrefillMxf };
 #ifndef MOE_MXF_DECODE
 #define MOE_MXF_DECODE 1
 #endif
-#ifndef MOE_DEC_LEGACY
-#define MOE_DEC_LEGACY 0
-#endif
+
 #ifndef MOE_MXF_PREFILL
 #define MOE_MXF_PREFILL 0
 #endif
@@ -496,17 +405,10 @@ bool config_fits(int64_t H, int64_t I) {
 
 // NVFP4 banks always take the converter kernel: the block-scaled MMA of the decode
 // tiles reads E8M0 scales per 32 elements only.
-bool dec_fits(int64_t H, int64_t I) {
-    if (MOE_DEC_LEGACY) return config_fits<moe::mxf::DecodeCfg>(H, I);
-    const int optin = max_smem_optin();
-    return H >= 128 && I >= 128 && (int)moe::dec::smem_bytes((int)(H / 32)) <= optin &&
-           (int)moe::dec::smem_bytes((int)(I / 32)) <= optin;
-}
-
 TileConfig pick_config(int64_t P, int64_t H, int64_t I, int64_t E, bool nv) {
     if (nv) return use_decode_tiles(P, E) ? kDecodeSmem : kPrefillSmem;
     if (use_decode_tiles(P, E))
-        return (MOE_MXF_DECODE && dec_fits(H, I)) ? kDecodeMxf : kDecodeSmem;
+        return (MOE_MXF_DECODE && config_fits<moe::mxf::DecodeCfg>(H, I)) ? kDecodeMxf : kDecodeSmem;
     return (MOE_MXF_PREFILL && config_fits<moe::mxf::PrefillCfg>(H, I)) ? kPrefillMxf : kPrefillSmem;
 }
 
@@ -587,10 +489,7 @@ int forward_layer(bool nv, const uint16_t *x, int64_t T, int64_t H, int64_t I, i
     float *yp = rows_out ? rows_out : reinterpret_cast<float *>(ws + L.yp);
 
     const int64_t P = T * k;
-    TileConfig cfg = pick_config(P, H, I, E, nv);
-    // the decode kernel's weight loads unpack 4-bit codes, which needs 32-byte aligned banks
-    if (cfg == kDecodeMxf && !MOE_DEC_LEGACY && (!aligned(gate_up_blocks, 32) || !aligned(down_blocks, 32)))
-        cfg = kDecodeSmem;
+    const TileConfig cfg = pick_config(P, H, I, E, nv);
     int rc = MOE_OK;
     do {
         if ((rc = launch_permute(ids, (int)expert_base, P, E, config_tok(cfg), counts, offsets, tile_offsets,
@@ -653,14 +552,15 @@ int launch_mxfp4_dequant(const uint8_t *blocks, const uint8_t *scales, uint16_t 
     if (!blocks || !scales || !out) return MOE_ERR_INVALID_ARG;
     if (E < 1 || N < 1 || K < 32 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
     if (!aligned(blocks, 16) || !aligned(out, 16)) return MOE_ERR_INVALID_ARG;
+    // one wave of 6 blocks per SM, each owning a contiguous run of whole rounds
     const int64_t n_words = E * N * (K / 8);
-    const int threads = 256;
-    int64_t blocks_needed = (n_words + threads - 1) / threads;
-    const int64_t cap = (int64_t)sm_count() * 8;
-    const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
+    const int64_t rounds = moe::ceil_div(n_words, moe::kDequantWords);
+    const int64_t cap = (int64_t)sm_count() * 6;
+    const int grid = (int)(rounds < cap ? rounds : cap);
+    const int64_t words_per_block = moe::ceil_div(rounds, grid) * moe::kDequantWords;
     StageScope scope(MOE_STAGE_DEQUANT, stream);
-    moe::mxfp4_dequant_kernel<kHostSrc><<<grid, threads, 0, stream>>>(
-        reinterpret_cast<const uint32_t *>(blocks), scales, reinterpret_cast<uint4 *>(out), n_words);
+    moe::mxfp4_dequant_kernel<kHostSrc><<<grid, moe::kDequantThreads, 0, stream>>>(
+        reinterpret_cast<const uint32_t *>(blocks), scales, reinterpret_cast<uint4 *>(out), n_words, words_per_block);
     return launch_check();
 }
 

@@ -270,26 +270,6 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
     return d;
 }
 
-// Shared-memory matrix descriptor for a K-major operand without swizzling: 8-row
-// core matrices of 16-byte rows, rows 16 B apart, core matrices 128 B apart along
-// M/N (a 32 x 16 B matrix is four core matrices, 512 contiguous bytes).
-__device__ __forceinline__ uint64_t plain_kmajor_desc(uint32_t smem_addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);   // start address
-    d |= (uint64_t)(128 >> 4) << 16;                 // leading byte offset
-    d |= (uint64_t)(128 >> 4) << 32;                 // stride byte offset: 8 rows x 16 B
-    d |= (uint64_t)1 << 46;                          // descriptor version for sm_100
-    return d;                                        // layout: no swizzle
-}
-
-// Asynchronous copy of a 32-row x 128-bit matrix from shared memory (descriptor) into
-// tensor memory at taddr (lane 0, four 32-bit columns), replicated into all four
-// lane quarters: lane l of every quarter receives row l.  Ordered with the MMAs the
-// same thread issues afterwards; completion is tracked by tcgen05.commit.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
-}
-
 // Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                      // D format fp32
