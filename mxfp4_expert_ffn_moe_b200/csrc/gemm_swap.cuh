@@ -195,6 +195,118 @@ __device__ __forceinline__ uint32_t e4m3_to_bf16x2(uint32_t b) {
     return h * 0x10001u;
 }
 
+// The epilogue of one work item, run by the four epilogue warps: TMEM accumulator
+// columns [acc, acc + ntok) of lane quarter q (weight rows 32 q .. 32 q + 31 of the
+// tile) -> the act rows (gate_up: bias, gate/up pairing, clamped SwiGLU, bf16) or
+// the yp rows (down: bias, routing weight, fp32).  stg is this warp's 4 KB of
+// shared-memory staging.
+template <int TOK, bool kGateUp, bool kNv>
+__device__ __forceinline__ void epilogue_tile(const Params &p, const Tile &t, uint32_t acc, uint8_t *stg_bytes,
+                                              int q, int lane) {
+    const int r = q * 32 + lane;             // weight row within the tile
+    const bool row_ok = r < t.mrows;
+    const int n = t.m0 + r;                             // output feature of this thread
+    const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
+    // NVFP4 weight_scale_2 of this row (gate rows are even), applied before the bias;
+    // the down projection's is one per expert and is loaded per chunk below
+    const float rs = (kNv && kGateUp && p.scale2 && row_ok) ? __ldg(p.scale2 + 2 * t.e + (n & 1)) : 1.0f;
+    // down: lane i holds the pair index and routing weight of token 32 j + i
+    int pairs[TOK / 32];
+    float wts[TOK / 32];
+    if (!kGateUp) {
+#pragma unroll
+        for (int j = 0; j < TOK / 32; ++j) {
+            const int tok = 32 * j + lane;
+            pairs[j] = (tok < t.ntok && in_bounds(t.row0 + tok, p.rows_cap)) ? __ldg(p.sorted_pairs + t.row0 + tok) : 0;
+            wts[j] = (tok < t.ntok && !p.weight_on_input) ? __ldg(p.weights + pairs[j]) : 1.0f;
+        }
+    }
+    for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+        const uint32_t taddr = acc + c0 + ((uint32_t)(q * 32) << 16);
+        uint32_t v[32];
+        if (kGateUp || !kNv) {
+            ptx::tmem_ld_32x32b_x32(taddr, v);
+            ptx::tmem_ld_wait();
+        }
+        const int nvalid = min(32, t.ntok - c0);
+        if (kGateUp) {
+            // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
+            // even lane finishes tokens 0..15 of the chunk, the odd lane 16..31.
+            // The warp's 16 features x 32 tokens go through a 1 KB staging tile
+            // so that every lane then stores whole 16-byte pieces of act rows.
+            const bool odd = lane & 1;
+            const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
+            const float bg = odd ? pb : bias, bu = odd ? bias : pb;
+            uint16_t *stg = reinterpret_cast<uint16_t *>(stg_bytes);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float lo_v = rs * __uint_as_float(v[i]), hi_v = rs * __uint_as_float(v[16 + i]);
+                const float mine = odd ? hi_v : lo_v;
+                const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? lo_v : hi_v, 1);
+                const float gate = (odd ? other : mine) + bg;
+                const float up = (odd ? mine : other) + bu;
+                const float a = clamped_swiglu(gate, up, p.alpha, p.limit);
+                stg[(odd ? 16 + i : i) * 16 + (lane >> 1)] = (uint16_t)(pack_bf16x2(a, 0.0f) & 0xFFFFu);
+            }
+            __syncwarp();
+            const int64_t fbase = (t.m0 + 32 * q) >> 1;     // first feature of the warp
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int piece = lane + 32 * h;            // 64 pieces of 16 bytes
+                const int tok = piece >> 1;
+                if (tok < nvalid && in_bounds(t.row0 + c0 + tok, p.rows_cap) &&
+                    range_in_bounds(fbase + (piece & 1) * 8, fbase + (piece & 1) * 8 + 8, p.N / 2)) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stg + tok * 16 + (piece & 1) * 8);
+                    *reinterpret_cast<uint4 *>(p.act + (int64_t)(t.row0 + c0 + tok) * (p.N / 2) +
+                                               fbase + (piece & 1) * 8) = val;
+                }
+            }
+            __syncwarp();
+        } else {
+            // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
+            // so that each pair's row segment leaves as 16-byte stores
+            float *stg = reinterpret_cast<float *>(stg_bytes);
+            if constexpr (kNv) {
+                // w * (s * acc + bias), s the expert's down weight_scale_2; the
+                // accumulator comes in two 16-column pieces (register budget)
+                const float ds = p.scale2 ? __ldg(p.scale2 + t.e) : 1.0f;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t u[16];
+                    ptx::tmem_ld_32x32b_x16(taddr + 16u * hf, u);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], 16 * hf + i);
+                        stg[(16 * hf + i) * 32 + lane] = wi * fmaf(ds, __uint_as_float(u[i]), bias);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], i);
+                    stg[i * 32 + lane] = wi * (__uint_as_float(v[i]) + bias);
+                }
+            }
+            __syncwarp();
+            if (32 * q < t.mrows) {                      // warp-uniform
+#pragma unroll
+                for (int rd = 0; rd < 8; ++rd) {
+                    const int piece = rd * 32 + lane;    // 32 tokens x 8 pieces of 16 B
+                    const int tok = piece >> 3, part = piece & 7;
+                    const int pi = __shfl_sync(0xFFFFFFFFu, pairs[c0 >> 5], tok);
+                    if (tok < nvalid && in_bounds(pi, p.rows_cap) &&
+                        range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
+                        const float4 val = *reinterpret_cast<const float4 *>(stg + tok * 32 + part * 4);
+                        *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
 template <class Cfg, bool kGateUp, bool kNv = false>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_mxfp4_swap_kernel(const __grid_constant__ CUtensorMap tmap_x,
@@ -328,114 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < kFirstConvWarp) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                  // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;             // weight row within the tile
         uint32_t local = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x, ++local) {
             const Tile t = decode_tile<TOK>(p, s_toff, item, w_tiles);
             const int b = local % Cfg::NACC;
             if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_full(b), (local / Cfg::NACC) & 1u))) break;
             ptx::tc_fence_after();
-            const bool row_ok = r < t.mrows;
-            const int n = t.m0 + r;                             // output feature of this thread
-            const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
-            // NVFP4 weight_scale_2 of this row (gate rows are even), applied before the bias;
-            // the down projection's is one per expert and is loaded per chunk below
-            const float rs = (kNv && kGateUp && p.scale2 && row_ok) ? __ldg(p.scale2 + 2 * t.e + (n & 1)) : 1.0f;
-            // down: lane i holds the pair index and routing weight of token 32 j + i
-            int pairs[TOK / 32];
-            float wts[TOK / 32];
-            if (!kGateUp) {
-#pragma unroll
-                for (int j = 0; j < TOK / 32; ++j) {
-                    const int tok = 32 * j + lane;
-                    pairs[j] = (tok < t.ntok && in_bounds(t.row0 + tok, p.rows_cap)) ? __ldg(p.sorted_pairs + t.row0 + tok) : 0;
-                    wts[j] = (tok < t.ntok && !p.weight_on_input) ? __ldg(p.weights + pairs[j]) : 1.0f;
-                }
-            }
-            for (int c0 = 0; c0 < t.ntok; c0 += 32) {
-                const uint32_t taddr = tmem_base + b * Cfg::ACC_STRIDE + c0 + ((uint32_t)(q * 32) << 16);
-                uint32_t v[32];
-                if (kGateUp || !kNv) {
-                    ptx::tmem_ld_32x32b_x32(taddr, v);
-                    ptx::tmem_ld_wait();
-                }
-                const int nvalid = min(32, t.ntok - c0);
-                if (kGateUp) {
-                    // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
-                    // even lane finishes tokens 0..15 of the chunk, the odd lane 16..31.
-                    // The warp's 16 features x 32 tokens go through a 1 KB staging tile
-                    // so that every lane then stores whole 16-byte pieces of act rows.
-                    const bool odd = lane & 1;
-                    const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
-                    const float bg = odd ? pb : bias, bu = odd ? bias : pb;
-                    uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + 4096 * q);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float lo_v = rs * __uint_as_float(v[i]), hi_v = rs * __uint_as_float(v[16 + i]);
-                        const float mine = odd ? hi_v : lo_v;
-                        const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? lo_v : hi_v, 1);
-                        const float gate = (odd ? other : mine) + bg;
-                        const float up = (odd ? mine : other) + bu;
-                        const float a = clamped_swiglu(gate, up, p.alpha, p.limit);
-                        stg[(odd ? 16 + i : i) * 16 + (lane >> 1)] = (uint16_t)(pack_bf16x2(a, 0.0f) & 0xFFFFu);
-                    }
-                    __syncwarp();
-                    const int64_t fbase = (t.m0 + 32 * q) >> 1;     // first feature of the warp
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int piece = lane + 32 * h;            // 64 pieces of 16 bytes
-                        const int tok = piece >> 1;
-                        if (tok < nvalid && in_bounds(t.row0 + c0 + tok, p.rows_cap) &&
-                            range_in_bounds(fbase + (piece & 1) * 8, fbase + (piece & 1) * 8 + 8, p.N / 2)) {
-                            const uint4 val = *reinterpret_cast<const uint4 *>(stg + tok * 16 + (piece & 1) * 8);
-                            *reinterpret_cast<uint4 *>(p.act + (int64_t)(t.row0 + c0 + tok) * (p.N / 2) +
-                                                       fbase + (piece & 1) * 8) = val;
-                        }
-                    }
-                    __syncwarp();
-                } else {
-                    // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
-                    // so that each pair's row segment leaves as 16-byte stores
-                    float *stg = reinterpret_cast<float *>(gbase + Cfg::OFF_EPI + 4096 * q);
-                    if constexpr (kNv) {
-                        // w * (s * acc + bias), s the expert's down weight_scale_2; the
-                        // accumulator comes in two 16-column pieces (register budget)
-                        const float ds = p.scale2 ? __ldg(p.scale2 + t.e) : 1.0f;
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            uint32_t u[16];
-                            ptx::tmem_ld_32x32b_x16(taddr + 16u * hf, u);
-                            ptx::tmem_ld_wait();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], 16 * hf + i);
-                                stg[(16 * hf + i) * 32 + lane] = wi * fmaf(ds, __uint_as_float(u[i]), bias);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float wi = __shfl_sync(0xFFFFFFFFu, wts[c0 >> 5], i);
-                            stg[i * 32 + lane] = wi * (__uint_as_float(v[i]) + bias);
-                        }
-                    }
-                    __syncwarp();
-                    if (32 * q < t.mrows) {                      // warp-uniform
-#pragma unroll
-                        for (int rd = 0; rd < 8; ++rd) {
-                            const int piece = rd * 32 + lane;    // 32 tokens x 8 pieces of 16 B
-                            const int tok = piece >> 3, part = piece & 7;
-                            const int pi = __shfl_sync(0xFFFFFFFFu, pairs[c0 >> 5], tok);
-                            if (tok < nvalid && in_bounds(pi, p.rows_cap) &&
-                                range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
-                                const float4 val = *reinterpret_cast<const float4 *>(stg + tok * 32 + part * 4);
-                                *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
-                            }
-                        }
-                    }
-                    __syncwarp();
-                }
-            }
+            epilogue_tile<TOK, kGateUp, kNv>(p, t, tmem_base + b * Cfg::ACC_STRIDE,
+                                             gbase + Cfg::OFF_EPI + 4096 * q, q, lane);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(a_empty(b));
