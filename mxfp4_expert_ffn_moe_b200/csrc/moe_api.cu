@@ -116,6 +116,27 @@ void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
     cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);   // errors surface in launch_check
 }
 
+// The same with thread-block clusters of `cluster` CTAs along x (grid.x a multiple).
+template <typename... KArgs, typename... Args>
+void launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, unsigned cluster,
+                        cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);   // errors surface in launch_check
+}
+
 // ---- per-stage launch counting and optional CUDA-event timing ---------------
 struct TimedLaunch {
     int stage;
@@ -716,14 +737,26 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
     const int slots = moe::rtr::ring_slots((int)E);
     const uint32_t smem = moe::rtr::smem_bytes((int)E, slots);
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
-    auto kernel = slots == 8 ? moe::rtr::router_route_kernel<8>
-                  : slots == 6 ? moe::rtr::router_route_kernel<6> : moe::rtr::router_route_kernel<4>;
+    // the split-K partials reuse the ring once the K loop is done
+    if (moe::rtr::partial_bytes((int)E) > (uint32_t)slots * moe::rtr::stage_bytes((int)E)) return MOE_ERR_UNSUPPORTED;
+    auto kernel = k <= 4 ? (slots == 8   ? moe::rtr::router_route_kernel<8, 4>
+                            : slots == 6 ? moe::rtr::router_route_kernel<6, 4>
+                                         : moe::rtr::router_route_kernel<4, 4>)
+                         : (slots == 8   ? moe::rtr::router_route_kernel<8, 8>
+                            : slots == 6 ? moe::rtr::router_route_kernel<6, 8>
+                                         : moe::rtr::router_route_kernel<4, 8>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MOE_ERR_CUDA;
-    const int64_t grid = moe::ceil_div(T, moe::rtr::BM);
+    // K split over a cluster of up to 8 CTAs per 128-token tile, so that small T still
+    // spreads over the SMs (and no split once the tiles alone fill them)
+    const int64_t tiles = moe::ceil_div(T, moe::rtr::BM);
+    // (a power of two: a token's threads are adjacent lanes of one warp)
+    int64_t ksplit = 1;
+    while (ksplit < 8 && tiles * ksplit * 2 <= sm_count() && ksplit * 2 <= H / moe::rtr::BK) ksplit *= 2;
+    if (tiles * ksplit > (int64_t)0x7FFFFFFF) return MOE_ERR_INVALID_ARG;
     StageScope scope(MOE_STAGE_ROUTE, s);
-    launch_pdl(kernel, dim3((unsigned)grid), dim3(moe::rtr::kThreads), smem, s, mx, mw, b_router, (int)T, (int)H,
-               (int)E, k, logits, ids, weights);
+    launch_pdl_cluster(kernel, dim3((unsigned)(tiles * ksplit)), dim3(moe::rtr::kThreads), smem, (unsigned)ksplit, s,
+                       mx, mw, b_router, (int)T, (int)H, (int)E, k, (int)ksplit, logits, ids, weights);
     return launch_check();
 }
 

@@ -59,8 +59,12 @@ def _check(moe, oracle, r, rows=None, bias=True):
     assert moe.moe_get_device_error() == 0
 
 
+# the K loop is split over clusters of 1, 2, 4 or 8 CTAs depending on T and H (8 for
+# few tiles and long K, 1 once the tiles fill the SMs: the last case); top-k lists of
+# 4 (k <= 4) and 8
 @pytest.mark.parametrize("T,H,E,k", [(1, 64, 4, 1), (37, 192, 32, 4), (130, 64, 7, 7), (300, 2880, 128, 4),
-                                     (5, 128, 256, 8), (129, 2880, 200, 8), (256, 448, 64, 2)])
+                                     (5, 128, 256, 8), (129, 2880, 200, 8), (256, 448, 64, 2),
+                                     (18949, 256, 8, 2)])
 def test_router_matches_oracle(moe_gpu, oracle_mod, T, H, E, k):
     _check(moe_gpu, oracle_mod, make_router(T, H, E, k, seed=T + E))
 
