@@ -214,6 +214,156 @@ __device__ __forceinline__ uint32_t mask_pad_blocks(uint32_t w, int kb0, int kbl
     return (w & keep) | (0x7F7F7F7Fu & ~keep);
 }
 
+// The epilogue of one decode work item, run by the four epilogue warps: accumulator
+// columns acc + [0, h) (hi terms) and acc + [h, 2h) (lo terms) of this warp's TMEM lane
+// quarter q -> the gate_up activation, written split as the next projection's B (block
+// maxima shared with the partner warp of the 32-feature block through `xch` and the
+// bounded barrier `xbar`), or the down rows of yp.  stg_bytes: this warp's 2 KB of
+// staging; `chunk` counts the warp's 32-token chunks (the exchange buffers alternate).
+// Returns false when a wait timed out.
+template <bool kGateUp>
+__device__ __forceinline__ bool epilogue_item(const Params &p, const Tile &t, uint32_t acc, uint8_t *stg_bytes,
+                                              float *xch, uint32_t xbar, uint32_t &chunk, int q, int lane) {
+    const int r = q * 32 + lane;             // weight row within the tile
+    bool ok = true;
+    const bool row_ok = r < t.mrows;
+    const int n = t.m0 + r;
+    const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
+        for (int c0 = 0; c0 < t.ntok; c0 += 32, ++chunk) {
+        // hi-term columns, then the lo-term columns added in two pieces of 16
+        // (keeps the live registers at 48)
+        uint32_t vh[32];
+        ptx::tmem_ld_32x32b_x32(acc + c0, vh);
+        ptx::tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vh[i]);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t vl[16];
+            ptx::tmem_ld_32x32b_x16(acc + t.h + c0 + 16 * hf, vl);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[16 * hf + i] += __uint_as_float(vl[i]);
+        }
+        const int nvalid = min(32, t.ntok - c0);
+        if (kGateUp) {
+            // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
+            // even lane finishes tokens 0..15 of the chunk, the odd lane 16..31,
+            // into a bf16 staging tile [token][16 features]
+            const bool odd = lane & 1;
+            const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
+            const float bg = odd ? pb : bias, bu = odd ? bias : pb;
+            uint16_t *stg = reinterpret_cast<uint16_t *>(stg_bytes);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float mine = odd ? v[16 + i] : v[i];
+                const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? v[i] : v[16 + i], 1);
+                const float gate = (odd ? other : mine) + bg;
+                const float up = (odd ? mine : other) + bu;
+                const float a = clamped_swiglu(gate, up, p.alpha, p.limit);
+                stg[(odd ? 16 + i : i) * 16 + (lane >> 1)] = (uint16_t)(pack_bf16x2(a, 0.0f) & 0xFFFFu);
+            }
+            __syncwarp();
+            // lane = token: its 16 features, the 32-feature block maximum shared
+            // with the partner warp (lane quarters 0/1 and 2/3 hold one block)
+            const uint4 s0 = *reinterpret_cast<const uint4 *>(stg + lane * 16);
+            const uint4 s1 = *reinterpret_cast<const uint4 *>(stg + lane * 16 + 8);
+            const uint32_t wv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(wv[i])), fabsf(bf16hi_to_f32(wv[i]))));
+            // double-buffered by chunk parity: a warp rewrites a buffer only after
+            // the handshake of the next chunk, which its partner joins after
+            // reading this one
+            float *xs = xch + (chunk & 1) * 128;
+            xs[q * 32 + lane] = amax;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(xbar);
+            ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(xbar, chunk & 1u)) && ok;
+            amax = fmaxf(amax, xs[(q ^ 1) * 32 + lane]);
+            const uint32_t bsc = split_scale_byte(amax);
+            uint32_t hq[4], lq[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t h0, l0, h1, l1;
+                split_pair(bf16lo_to_f32(wv[2 * i]), bf16hi_to_f32(wv[2 * i]), bsc, h0, l0);
+                split_pair(bf16lo_to_f32(wv[2 * i + 1]), bf16hi_to_f32(wv[2 * i + 1]), bsc, h1, l1);
+                hq[i] = h0 | (h1 << 16);
+                lq[i] = l0 | (l1 << 16);
+            }
+            const int I = p.N / 2;
+            const int64_t RS = split_row_bytes(I);
+            const int f0 = (t.m0 >> 1) + 16 * q;     // first feature of this warp
+            if (lane < nvalid && f0 < I && in_bounds(t.row0 + c0 + lane, p.P) &&
+                range_in_bounds(f0, f0 + 16, I)) {
+                const int64_t row = t.row0 + c0 + lane;
+                uint8_t *hrow = p.actq + row * RS;
+                uint8_t *lrow = p.actq + ((int64_t)p.P + row) * RS;
+                *reinterpret_cast<uint4 *>(hrow + f0) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+                *reinterpret_cast<uint4 *>(lrow + f0) = make_uint4(lq[0], lq[1], lq[2], lq[3]);
+                if ((q & 1) == 0) {   // one warp of the pair writes the block's scale bytes
+                    const int blk = f0 >> 5;
+                    const int64_t slot = I + 16 * (blk >> 2);
+                    hrow[slot + (blk & 3)] = (uint8_t)bsc;
+                    lrow[slot + (blk & 3)] = (uint8_t)(bsc - 4u);
+                    if ((blk & 3) == 0) {
+                        // the writer of a step's first block completes the slot the
+                        // way the token split does: scale 1 (127) for blocks past I,
+                        // zeros after the scale word, so no byte of the slot is left
+                        // from an earlier call
+                        const int nblk = I / 32;
+#pragma unroll
+                        for (int j = 1; j < 4; ++j)
+                            if (blk + j >= nblk) hrow[slot + j] = lrow[slot + j] = 127u;
+                        uint32_t *hw = reinterpret_cast<uint32_t *>(hrow + slot);
+                        uint32_t *lw = reinterpret_cast<uint32_t *>(lrow + slot);
+                        hw[1] = hw[2] = hw[3] = 0u;
+                        lw[1] = lw[2] = lw[3] = 0u;
+                    }
+                }
+            }
+            __syncwarp();
+        } else {
+            // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
+            // so that each pair's row segment leaves as 16-byte stores
+            int pair_l = 0;
+            float wt_l = 1.0f;
+            if (lane < nvalid && in_bounds(t.row0 + c0 + lane, p.P)) {
+                pair_l = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
+                if (!p.weight_on_input) wt_l = __ldg(p.weights + pair_l);
+            }
+            // two passes of 16 tokens through a 2 KB staging tile
+            float *stg = reinterpret_cast<float *>(stg_bytes);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float wi = __shfl_sync(0xFFFFFFFFu, wt_l, 16 * hf + i);
+                    stg[i * 32 + lane] = wi * (v[16 * hf + i] + bias);
+                }
+                __syncwarp();
+                if (32 * q < t.mrows) {                  // warp-uniform
+#pragma unroll
+                    for (int rd = 0; rd < 4; ++rd) {
+                        const int piece = rd * 32 + lane;    // 16 tokens x 8 pieces of 16 B
+                        const int tok = 16 * hf + (piece >> 3), part = piece & 7;
+                        const int pi = __shfl_sync(0xFFFFFFFFu, pair_l, tok);
+                        if (tok < nvalid && in_bounds(pi, p.P) &&
+                            range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
+                            const float4 val = *reinterpret_cast<const float4 *>(stg + (piece >> 3) * 32 + part * 4);
+                            *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+    return ok;
+}
+
 template <class Cfg, bool kGateUp>
 __global__ void __launch_bounds__(Cfg::kThreads, 1)
     grouped_mxfp4_mxf_kernel(const __grid_constant__ CUtensorMap tmap_b,
@@ -386,7 +536,6 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
     } else if (warp < kFirstStageWarp) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;                  // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;             // weight row within the tile
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         float *const xch = reinterpret_cast<float *>(gbase + Cfg::OFF_XCH);
         uint32_t local = 0, chunk = 0;
@@ -396,142 +545,9 @@ __global__ void __launch_bounds__(Cfg::kThreads, 1)
             const int b = local % NACC;
             if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(a_full(b), (local / NACC) & 1u))) break;
             ptx::tc_fence_after();
-            const bool row_ok = r < t.mrows;
-            const int n = t.m0 + r;
-            const float bias = (p.bias && row_ok) ? __ldg(p.bias + (int64_t)t.e * p.N + n) : 0.0f;
-            const uint32_t acc = tmem_base + b * Cfg::ACC_COLS + lane_off;
-            for (int c0 = 0; c0 < t.ntok; c0 += 32, ++chunk) {
-                // hi-term columns, then the lo-term columns added in two pieces of 16
-                // (keeps the live registers at 48)
-                uint32_t vh[32];
-                ptx::tmem_ld_32x32b_x32(acc + c0, vh);
-                ptx::tmem_ld_wait();
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vh[i]);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t vl[16];
-                    ptx::tmem_ld_32x32b_x16(acc + t.h + c0 + 16 * hf, vl);
-                    ptx::tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[16 * hf + i] += __uint_as_float(vl[i]);
-                }
-                const int nvalid = min(32, t.ntok - c0);
-                if (kGateUp) {
-                    // lanes 2i (gate row) and 2i+1 (up row) hold one output feature; the
-                    // even lane finishes tokens 0..15 of the chunk, the odd lane 16..31,
-                    // into a bf16 staging tile [token][16 features]
-                    const bool odd = lane & 1;
-                    const float pb = __shfl_xor_sync(0xFFFFFFFFu, bias, 1);
-                    const float bg = odd ? pb : bias, bu = odd ? bias : pb;
-                    uint16_t *stg = reinterpret_cast<uint16_t *>(gbase + Cfg::OFF_EPI + kEpiStage * q);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float mine = odd ? v[16 + i] : v[i];
-                        const float other = __shfl_xor_sync(0xFFFFFFFFu, odd ? v[i] : v[16 + i], 1);
-                        const float gate = (odd ? other : mine) + bg;
-                        const float up = (odd ? mine : other) + bu;
-                        const float a = clamped_swiglu(gate, up, p.alpha, p.limit);
-                        stg[(odd ? 16 + i : i) * 16 + (lane >> 1)] = (uint16_t)(pack_bf16x2(a, 0.0f) & 0xFFFFu);
-                    }
-                    __syncwarp();
-                    // lane = token: its 16 features, the 32-feature block maximum shared
-                    // with the partner warp (lane quarters 0/1 and 2/3 hold one block)
-                    const uint4 s0 = *reinterpret_cast<const uint4 *>(stg + lane * 16);
-                    const uint4 s1 = *reinterpret_cast<const uint4 *>(stg + lane * 16 + 8);
-                    const uint32_t wv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        amax = fmaxf(amax, fmaxf(fabsf(bf16lo_to_f32(wv[i])), fabsf(bf16hi_to_f32(wv[i]))));
-                    // double-buffered by chunk parity: a warp rewrites a buffer only after
-                    // the handshake of the next chunk, which its partner joins after
-                    // reading this one
-                    float *xs = xch + (chunk & 1) * 128;
-                    xs[q * 32 + lane] = amax;
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(xch_bar(q >> 1));
-                    ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(xch_bar(q >> 1), chunk & 1u));
-                    amax = fmaxf(amax, xs[(q ^ 1) * 32 + lane]);
-                    const uint32_t bsc = split_scale_byte(amax);
-                    uint32_t hq[4], lq[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t h0, l0, h1, l1;
-                        split_pair(bf16lo_to_f32(wv[2 * i]), bf16hi_to_f32(wv[2 * i]), bsc, h0, l0);
-                        split_pair(bf16lo_to_f32(wv[2 * i + 1]), bf16hi_to_f32(wv[2 * i + 1]), bsc, h1, l1);
-                        hq[i] = h0 | (h1 << 16);
-                        lq[i] = l0 | (l1 << 16);
-                    }
-                    const int I = p.N / 2;
-                    const int64_t RS = split_row_bytes(I);
-                    const int f0 = (t.m0 >> 1) + 16 * q;     // first feature of this warp
-                    if (lane < nvalid && f0 < I && in_bounds(t.row0 + c0 + lane, p.P) &&
-                        range_in_bounds(f0, f0 + 16, I)) {
-                        const int64_t row = t.row0 + c0 + lane;
-                        uint8_t *hrow = p.actq + row * RS;
-                        uint8_t *lrow = p.actq + ((int64_t)p.P + row) * RS;
-                        *reinterpret_cast<uint4 *>(hrow + f0) = make_uint4(hq[0], hq[1], hq[2], hq[3]);
-                        *reinterpret_cast<uint4 *>(lrow + f0) = make_uint4(lq[0], lq[1], lq[2], lq[3]);
-                        if ((q & 1) == 0) {   // one warp of the pair writes the block's scale bytes
-                            const int blk = f0 >> 5;
-                            const int64_t slot = I + 16 * (blk >> 2);
-                            hrow[slot + (blk & 3)] = (uint8_t)bsc;
-                            lrow[slot + (blk & 3)] = (uint8_t)(bsc - 4u);
-                            if ((blk & 3) == 0) {
-                                // the writer of a step's first block completes the slot the
-                                // way the token split does: scale 1 (127) for blocks past I,
-                                // zeros after the scale word, so no byte of the slot is left
-                                // from an earlier call
-                                const int nblk = I / 32;
-#pragma unroll
-                                for (int j = 1; j < 4; ++j)
-                                    if (blk + j >= nblk) hrow[slot + j] = lrow[slot + j] = 127u;
-                                uint32_t *hw = reinterpret_cast<uint32_t *>(hrow + slot);
-                                uint32_t *lw = reinterpret_cast<uint32_t *>(lrow + slot);
-                                hw[1] = hw[2] = hw[3] = 0u;
-                                lw[1] = lw[2] = lw[3] = 0u;
-                            }
-                        }
-                    }
-                    __syncwarp();
-                } else {
-                    // w * (acc + bias) for 32 tokens x the warp's 32 features, staged
-                    // so that each pair's row segment leaves as 16-byte stores
-                    int pair_l = 0;
-                    float wt_l = 1.0f;
-                    if (lane < nvalid && in_bounds(t.row0 + c0 + lane, p.P)) {
-                        pair_l = __ldg(p.sorted_pairs + t.row0 + c0 + lane);
-                        if (!p.weight_on_input) wt_l = __ldg(p.weights + pair_l);
-                    }
-                    // two passes of 16 tokens through a 2 KB staging tile
-                    float *stg = reinterpret_cast<float *>(gbase + Cfg::OFF_EPI + kEpiStage * q);
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float wi = __shfl_sync(0xFFFFFFFFu, wt_l, 16 * hf + i);
-                            stg[i * 32 + lane] = wi * (v[16 * hf + i] + bias);
-                        }
-                        __syncwarp();
-                        if (32 * q < t.mrows) {                  // warp-uniform
-#pragma unroll
-                            for (int rd = 0; rd < 4; ++rd) {
-                                const int piece = rd * 32 + lane;    // 16 tokens x 8 pieces of 16 B
-                                const int tok = 16 * hf + (piece >> 3), part = piece & 7;
-                                const int pi = __shfl_sync(0xFFFFFFFFu, pair_l, tok);
-                                if (tok < nvalid && in_bounds(pi, p.P) &&
-                                    range_in_bounds(t.m0 + 32 * q + part * 4, t.m0 + 32 * q + part * 4 + 4, p.N)) {
-                                    const float4 val = *reinterpret_cast<const float4 *>(stg + (piece >> 3) * 32 + part * 4);
-                                    *reinterpret_cast<float4 *>(p.yp + (int64_t)pi * p.N + t.m0 + 32 * q + part * 4) = val;
-                                }
-                            }
-                        }
-                        __syncwarp();
-                    }
-                }
-            }
+            ok = epilogue_item<kGateUp>(p, t, tmem_base + b * Cfg::ACC_COLS + lane_off,
+                                        gbase + Cfg::OFF_EPI + kEpiStage * q, xch, xch_bar(q >> 1), chunk, q,
+                                        lane);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(a_empty(b));
