@@ -7,6 +7,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <tuple>
 #include <utility>
 #include <vector>
 
@@ -16,6 +19,7 @@
 #include <stdlib.h>
 
 #include "../../include/moe_mxfp4.h"
+#include "context_id.h"
 #include "combine.cuh"
 #include "common.cuh"
 #include "dequant.cuh"
@@ -262,6 +266,33 @@ bool make_packed_map(CUtensorMap *m, const void *ptr, int64_t E, int64_t N, int6
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) is a driver call per function and
+// context; the largest size already set is remembered per (kernel, device, context), so
+// that repeated calls of an entry point skip it (a new context is a miss).
+bool ensure_smem_attr(const void *kernel, int bytes) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int, unsigned long long>, int> done;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const unsigned long long ctx = moe::current_context_id();
+    const auto key = std::make_tuple(kernel, dev, ctx);
+    if (ctx != 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = done.find(key);
+        if (it != done.end() && it->second >= bytes) return true;
+    }
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (ctx != 0) {
+        std::lock_guard<std::mutex> lock(mu);
+        int &v = done[key];
+        if (v < bytes) v = bytes;
+    }
+    return true;
+}
+
 int max_smem_optin() {
     int dev = 0, v = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -301,7 +332,7 @@ int launch_grouped_gemm(int stage, const uint16_t *A, int64_t rows, int64_t K, c
     const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
     auto kernel = moe::swp::grouped_mxfp4_swap_kernel<Cfg, kGateUp, kNv>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(kernel), (int)smem))
         return MOE_ERR_CUDA;
     const int64_t w_tiles = moe::ceil_div(N, moe::swp::BM);
     const int64_t max_items = (moe::ceil_div(rows, Cfg::TOK) + E) * w_tiles;
@@ -364,7 +395,7 @@ int launch_mxf_gemm(int stage, const uint8_t *bq, int64_t P, int64_t K, const ui
     const uint32_t smem = Cfg::smem_bytes((int)(K / 32));
     if ((int)smem > max_smem_optin()) return MOE_ERR_UNSUPPORTED;
     auto kernel = moe::mxf::grouped_mxfp4_mxf_kernel<Cfg, kGateUp>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(kernel), (int)smem))
         return MOE_ERR_CUDA;
     const int64_t w_tiles = moe::ceil_div(N, moe::mxf::BM);
     const int64_t max_items = (moe::ceil_div(P, Cfg::TOK) + E) * w_tiles;
@@ -443,14 +474,12 @@ int config_tok(TileConfig c) {
 }
 
 // Pair permutation (one CTA).  The ids are staged in shared memory when they fit (up
-// to ~50K pairs); the attribute is per device, so it is set on every call, like the
-// GEMMs'.
+// to ~50K pairs).
 int launch_permute(const int32_t *ids, int expert_base, int64_t P, int64_t E, int tile_rows, int32_t *counts,
                    int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
                    cudaStream_t s) {
-    const bool perm_attr = cudaFuncSetAttribute(moe::permute_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                (int)moe::kPermuteSmemCap) == cudaSuccess;
-    if (!perm_attr) cudaGetLastError();
+    const bool perm_attr = ensure_smem_attr(reinterpret_cast<const void *>(moe::permute_pairs_kernel),
+                                            (int)moe::kPermuteSmemCap);
     const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
     const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
     StageScope sp(MOE_STAGE_PERMUTE, s);
@@ -745,7 +774,7 @@ int moe_router_route(const uint16_t *x, const uint16_t *w_router, const float *b
                          : (slots == 8   ? moe::rtr::router_route_kernel<8, 8>
                             : slots == 6 ? moe::rtr::router_route_kernel<6, 8>
                                          : moe::rtr::router_route_kernel<4, 8>);
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(kernel), (int)smem))
         return MOE_ERR_CUDA;
     // K split over a cluster of up to 8 CTAs per 128-token tile, so that small T still
     // spreads over the SMs (and no split once the tiles alone fill them)

@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "../../include/moe_mxfp4.h"
+#include "context_id.h"
 
 // Held by every GPU that loads this library, until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
@@ -35,35 +36,6 @@ struct ScratchAddr {
 std::mutex g_scratch_mutex;
 ScratchAddr g_scratch[kMaxDevices] = {};
 
-// Identifier of the calling thread's current context, or 0 when there is none or
-// the driver entry points are unavailable (then every call looks the address up).
-// Called with g_scratch_mutex held.
-unsigned long long current_context_id() {
-    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
-    static PFN_cuCtxGetId_v12000 get_id = nullptr;
-    static bool resolved = false;
-    if (!resolved) {
-        void *a = nullptr, *b = nullptr;
-        cudaDriverEntryPointQueryResult qa, qb;
-        const bool ok_a = cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
-                          qa == cudaDriverEntryPointSuccess;
-        const bool ok_b = cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
-                          qb == cudaDriverEntryPointSuccess;
-        if (ok_a && ok_b) {
-            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
-            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
-        } else {
-            cudaGetLastError();
-        }
-        resolved = true;
-    }
-    if (!get_current || !get_id) return 0;
-    CUcontext ctx = nullptr;
-    unsigned long long id = 0;
-    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
-    return id;
-}
-
 // Device address of the scratch array on the current device, looked up on the
 // first call in each context of the device.
 int scratch_address(void **addr) {
@@ -71,7 +43,7 @@ int scratch_address(void **addr) {
     if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    const unsigned long long ctx = current_context_id();
+    const unsigned long long ctx = moe::current_context_id();
     if (ctx != 0 && g_scratch[dev].addr && g_scratch[dev].ctx_id == ctx) {
         *addr = g_scratch[dev].addr;
         return MOE_OK;
@@ -83,7 +55,7 @@ int scratch_address(void **addr) {
         return MOE_ERR_CUDA;
     }
     // the lookup has made the device's context current if it was not yet
-    g_scratch[dev] = ScratchAddr{current_context_id(), p};
+    g_scratch[dev] = ScratchAddr{moe::current_context_id(), p};
     *addr = p;
     return MOE_OK;
 }
