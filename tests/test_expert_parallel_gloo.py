@@ -123,14 +123,12 @@ def _rank(rank, world, port, woi, q):
     dist.destroy_process_group()
 
 
-@pytest.mark.timeout(240)
-@pytest.mark.parametrize("woi", [False, True], ids=["weight_on_output", "weight_on_input"])
-def test_two_rank_expert_parallel_equals_single_rank_oracle(woi):
+def _run_world(world, woi):
     import torch.multiprocessing as mp
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, woi, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, woi, q)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -139,12 +137,25 @@ def test_two_rank_expert_parallel_equals_single_rank_oracle(woi):
         if p.is_alive():
             p.kill()
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
-    res = sorted(q.get(timeout=10) for _ in range(2))
+    res = sorted(q.get(timeout=10) for _ in range(world))
     for rank, equal, maxdiff, sends_ok, recv_ok, nrecv in res:
         assert equal, (rank, maxdiff)
         assert sends_ok and recv_ok, rank
-    # every valid pair of both ranks was computed exactly once (14 tokens x 2 slots, one dropped)
-    assert sum(r[5] for r in res) == 2 * 7 * 2 - 1
+    # every valid pair of every rank was computed exactly once (7 tokens x 2 slots per
+    # rank, one dropped on rank 1)
+    assert sum(r[5] for r in res) == world * 7 * 2 - 1
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("woi", [False, True], ids=["weight_on_output", "weight_on_input"])
+def test_two_rank_expert_parallel_equals_single_rank_oracle(woi):
+    _run_world(2, woi)
+
+
+@pytest.mark.timeout(240)
+def test_three_rank_expert_parallel_with_uneven_ranges():
+    # 5 experts over 3 ranks: ranges of 1, 2 and 2 experts
+    _run_world(3, False)
 
 
 def test_expert_ranges_and_rows_per_rank():
