@@ -34,8 +34,8 @@ DEFAULT_WORKLOAD = "20b_prefill_T4096"
 # DRAM bytes (read + write) of one gate_up launch of the default workload, measured by
 # ncu (dram__bytes_read.sum + dram__bytes_write.sum) on the kernel whose source has the
 # SHA-256 prefix below; reported only while the source still matches, else null.
-GATE_UP_DRAM_BYTES = 464.9e6
-GATE_UP_SOURCE_SHA = "9adf60a72aca2c71"
+GATE_UP_DRAM_BYTES = 469.6e6
+GATE_UP_SOURCE_SHA = "e44c8fabd3ce3bff"
 GATE_UP_SOURCE = os.path.join(ROOT, "mxfp4_expert_ffn_moe_b200", "csrc", "gemm_swap.cuh")
 
 

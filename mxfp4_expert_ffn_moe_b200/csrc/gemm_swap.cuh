@@ -461,7 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 2^(s-1) (two, by 2^126 and 2^(s-127), when 2^(s-1) is not a bf16) gives
         // E2M1 * 2^(s-127) exactly; the result goes to the 128-byte swizzled
         // K-major layout the MMA reads.  The E8M0 bytes a thread needs for its
-        // group's next step are loaded from global memory one step ahead.
+        // group's next step are loaded from global memory one step ahead, and the
+        // next step is converted into registers while the MMA still reads the slot.
         // NVFP4: a block's two E4M3 bytes (one per 16 elements) come as one 16-bit
         // load; the codes are multiplied by 2^126 (exact E2M1) and then by the
         // E4M3 scale of their half as a bf16 (exact products).
@@ -493,32 +494,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // first step of this tile that belongs to this group
             int kb = (int)((grp - (int)(it % kConvGroups) + kConvGroups) % kConvGroups);
-            uint32_t nxt[kBlocksPerThread];
+            uint32_t nxt[kBlocksPerThread];     // scale bits of the next step to decode
 #pragma unroll
             for (int bi = 0; bi < kBlocksPerThread; ++bi)
                 nxt[bi] = (rok[bi] && kb < k_iters) ? load_sc(bi, kb) : kOne;
-            for (; kb < k_iters; kb += kConvGroups) {
-                const uint32_t gi = it + (uint32_t)kb;         // global step index
-                const int c = gi % S, ps = gi % PS;
-                uint32_t cur[kBlocksPerThread];
-#pragma unroll
-                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
-                    cur[bi] = nxt[bi];
-                    nxt[bi] = (rok[bi] && kb + kConvGroups < k_iters) ? load_sc(bi, kb + kConvGroups) : kOne;
-                }
-                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (gi / PS) & 1u)))) break;
-                uint4 q4[kBlocksPerThread];
+            // The group's steps are software-pipelined: step kb + kConvGroups is decoded
+            // into registers as soon as step kb is stored, so that once a stage slot is
+            // free only the stores remain.
+            uint32_t cv[kBlocksPerThread][16];
+            auto decode_step = [&](int kbi) -> bool {
+                const uint32_t gix = it + (uint32_t)kbi;
+                const int ps = gix % PS;
+                if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(wp_full(ps), (gix / PS) & 1u))) return false;
 #pragma unroll
                 for (int bi = 0; bi < kBlocksPerThread; ++bi) {
                     const int blkid = gt + bi * kGroupThreads;
-                    q4[bi] = ptx::ld_shared_v4(wp_stage(ps) + (blkid >> 1) * 32 + (blkid & 1) * 16);
-                }
-                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(c), ((gi / S) & 1u) ^ 1u)))) break;
-#pragma unroll
-                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
-                    const int blkid = gt + bi * kGroupThreads;    // 0 .. 255 within the step
-                    const int row = blkid >> 1, blk = blkid & 1;
-                    const uint32_t sc = cur[bi];
+                    const uint4 q4 = ptx::ld_shared_v4(wp_stage(ps) + (blkid >> 1) * 32 + (blkid & 1) * 16);
+                    const uint32_t sc = nxt[bi];
                     uint32_t m1, m2 = 0, m2b = 0;   // m2: words 0-1 (first 16 elements), m2b: words 2-3
                     if (kNv) {
                         m1 = 0x7E807E80u;
@@ -534,9 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         m2 = (sc << 7) * 0x10001u;
                     }
                     if (!kNv) m2b = m2;
-                    const uint32_t qw[4] = {q4[bi].x, q4[bi].y, q4[bi].z, q4[bi].w};
-                    const uint32_t dst_row = wb_stage(c) + row * 128;
-                    const uint32_t sw = (uint32_t)(row & 7);
+                    const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         uint32_t r0, r1, r2, r3;
@@ -552,18 +542,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                             r2 = ptx::hmul2_bf16(r2, mw);
                             r3 = ptx::hmul2_bf16(r3, mw);
                         }
+                        cv[bi][4 * w] = r0;
+                        cv[bi][4 * w + 1] = r1;
+                        cv[bi][4 * w + 2] = r2;
+                        cv[bi][4 * w + 3] = r3;
+                    }
+                }
+                // every lane has consumed its packed words, so the TMA may refill the slot
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(wp_empty(ps));
+#pragma unroll
+                for (int bi = 0; bi < kBlocksPerThread; ++bi)
+                    nxt[bi] = (rok[bi] && kbi + kConvGroups < k_iters) ? load_sc(bi, kbi + kConvGroups) : kOne;
+                return true;
+            };
+            if (kb < k_iters) ok = decode_step(kb);
+            for (; kb < k_iters && ok; kb += kConvGroups) {
+                const uint32_t gi = it + (uint32_t)kb;         // global step index
+                const int c = gi % S;
+                if (!(ok = __all_sync(0xFFFFFFFFu, ptx::mbar_wait(empty(c), ((gi / S) & 1u) ^ 1u)))) break;
+#pragma unroll
+                for (int bi = 0; bi < kBlocksPerThread; ++bi) {
+                    const int blkid = gt + bi * kGroupThreads;    // 0 .. 255 within the step
+                    const int row = blkid >> 1, blk = blkid & 1;
+                    const uint32_t dst_row = wb_stage(c) + row * 128;
+                    const uint32_t sw = (uint32_t)(row & 7);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
                         const uint32_t chunk = (uint32_t)(blk * 4 + w);
-                        ptx::st_shared_v4(dst_row + ((chunk ^ sw) << 4), r0, r1, r2, r3);
+                        ptx::st_shared_v4(dst_row + ((chunk ^ sw) << 4), cv[bi][4 * w], cv[bi][4 * w + 1],
+                                          cv[bi][4 * w + 2], cv[bi][4 * w + 3]);
                     }
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(ready(c));
-                    // every lane has consumed its packed words (the conversion used
-                    // them), so the TMA may refill the packed slot
-                    ptx::mbar_arrive(wp_empty(ps));
-                }
+                if (lane == 0) ptx::mbar_arrive(ready(c));
+                if (kb + kConvGroups < k_iters) ok = decode_step(kb + kConvGroups);
             }
             it += (uint32_t)k_iters;
         }
