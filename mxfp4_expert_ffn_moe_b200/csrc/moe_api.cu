@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -473,14 +474,14 @@ int config_tok(TileConfig c) {
     }
 }
 
-// Pair permutation (one CTA).  The ids are staged in shared memory when they fit (up
-// to ~50K pairs).
+// Pair permutation (one CTA).  The ids and the placed pairs are staged in shared
+// memory when they fit (up to ~35K pairs).
 int launch_permute(const int32_t *ids, int expert_base, int64_t P, int64_t E, int tile_rows, int32_t *counts,
                    int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
                    cudaStream_t s) {
-    const bool perm_attr = ensure_smem_attr(reinterpret_cast<const void *>(moe::permute_pairs_kernel),
-                                            (int)moe::kPermuteSmemCap);
-    const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= moe::kPermuteSmemCap;
+    const size_t cap = std::min<size_t>(moe::kPermuteSmemCap, (size_t)max_smem_optin());
+    const bool perm_attr = ensure_smem_attr(reinterpret_cast<const void *>(moe::permute_pairs_kernel), (int)cap);
+    const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= cap;
     const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
     StageScope sp(MOE_STAGE_PERMUTE, s);
     launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, expert_base, P,

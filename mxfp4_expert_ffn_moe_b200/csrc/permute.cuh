@@ -13,10 +13,13 @@
 //
 // One CTA of 32 warps: warp w owns a contiguous chunk of pairs, counts its experts
 // in a private shared-memory row, the chunk bases come from an exclusive scan over
-// warps, and each warp then scatters its chunk in order using __match_any_sync to
-// rank equal experts inside a 32-pair step.  When the ids fit (staged != 0) they are
-// first copied into shared memory with independent, coalesced loads, so neither
-// pass over them waits on a global load per step.
+// warps (the expert starts from one warp's shuffle scan), and each warp then places
+// its chunk in order using __match_any_sync to rank equal experts inside a 32-pair
+// step.  When they fit (staged != 0, up to ~35K pairs), the ids are first copied
+// into shared memory as 16-bit expert numbers with coalesced 16-byte loads, the pairs
+// are placed into a shared-memory copy of sorted_pairs, and that copy leaves with
+// coalesced 16-byte stores: one SM alone would otherwise issue one L2 transaction per
+// pair for the scattered stores.
 #pragma once
 #include "common.cuh"
 
@@ -24,12 +27,16 @@ namespace moe {
 
 constexpr int kPermuteThreads = 1024;
 
-// Dynamic shared memory of permute_pairs_kernel: the count rows and expert starts,
-// plus P staged ids when `staged`.
-__host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t P, bool staged) {
-    return sizeof(int) * (size_t)(32 * E + E + 1) + (staged ? sizeof(int) * (size_t)P : 0);
+// Dynamic shared memory of permute_pairs_kernel: the count rows and expert starts;
+// when staged, also the P ids (int16) and the P placed pairs (int32, 16-byte aligned).
+__host__ __device__ constexpr size_t permute_ids_offset(int E) { return sizeof(int) * (size_t)(33 * E + 1); }
+__host__ __device__ constexpr size_t permute_sorted_offset(int E, int64_t P) {
+    return (permute_ids_offset(E) + 2 * (size_t)P + 15) & ~(size_t)15;
 }
-constexpr size_t kPermuteSmemCap = 200 * 1024;
+__host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t P, bool staged) {
+    return staged ? permute_sorted_offset(E, P) + 4 * (size_t)P : permute_ids_offset(E);
+}
+constexpr size_t kPermuteSmemCap = 227 * 1024;
 
 __device__ __forceinline__ int relative_expert(int32_t id, int expert_base, int E) {
     const int64_t e = (int64_t)id - expert_base;
@@ -45,17 +52,40 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
     int32_t *__restrict__ sorted_pairs, int32_t *__restrict__ pair_rows) {
     pdl_wait();
     pdl_trigger();
-    extern __shared__ int sm_perm[];
-    int *cnt = sm_perm;             // [32][E]: per-warp counts, then per-warp running bases
-    int *off = sm_perm + 32 * E;    // [E + 1]: expert start rows
-    int *ids_s = off + E + 1;       // [P] when staged
+    extern __shared__ __align__(16) unsigned char sm_perm_raw[];
+    int *cnt = reinterpret_cast<int *>(sm_perm_raw);     // [32][E]: per-warp counts, then running bases
+    int *off = cnt + 32 * E;                              // [E + 1]: expert start rows
+    int16_t *ids_s = reinterpret_cast<int16_t *>(sm_perm_raw + permute_ids_offset(E));          // [P]
+    int32_t *sorted_s = reinterpret_cast<int32_t *>(sm_perm_raw + permute_sorted_offset(E, P));  // [P]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
-    if (staged)
-        for (int64_t i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = relative_expert(__ldg(ids + i), expert_base, E);
+    if (staged) {
+        // 16-byte loads, eight per thread in flight before their stores
+        const int64_t nv = ((reinterpret_cast<uintptr_t>(ids) & 15u) == 0) ? P / 4 : 0;
+        const int4 *ids4 = reinterpret_cast<const int4 *>(ids);
+        for (int64_t i0 = threadIdx.x; i0 < nv; i0 += 8 * (int64_t)blockDim.x) {
+            int4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * (int64_t)blockDim.x < nv) v[u] = __ldg(ids4 + i0 + u * (int64_t)blockDim.x);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t i = i0 + u * (int64_t)blockDim.x;
+                if (i >= nv) continue;
+                ids_s[4 * i] = (int16_t)relative_expert(v[u].x, expert_base, E);
+                ids_s[4 * i + 1] = (int16_t)relative_expert(v[u].y, expert_base, E);
+                ids_s[4 * i + 2] = (int16_t)relative_expert(v[u].z, expert_base, E);
+                ids_s[4 * i + 3] = (int16_t)relative_expert(v[u].w, expert_base, E);
+            }
+        }
+        for (int64_t i = 4 * nv + threadIdx.x; i < P; i += blockDim.x)
+            ids_s[i] = (int16_t)relative_expert(__ldg(ids + i), expert_base, E);
+    }
     __syncthreads();
     // expert of pair p relative to expert_base, -1 when outside [0, E)
-    auto expert_of = [&](int64_t p) { return staged ? ids_s[p] : relative_expert(__ldg(ids + p), expert_base, E); };
+    auto expert_of = [&](int64_t p) {
+        return staged ? (int)ids_s[p] : relative_expert(__ldg(ids + p), expert_base, E);
+    };
 
     const int64_t chunk = (P + 31) / 32;
     const int64_t beg = (int64_t)warp * chunk;
@@ -78,9 +108,27 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
         off[e] = run;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0, trun = 0;
-        for (int e = 0; e < E; ++e) {
+    if (warp == 0) {
+        // lane l takes experts [l*per, l*per + per): its totals, an exclusive scan of
+        // those over the lanes, then its experts' starts in order
+        const int per = (E + 31) / 32;
+        const int e0 = lane * per, e1 = min(e0 + per, E);
+        int sum = 0, tsum = 0;
+        for (int e = e0; e < e1; ++e) {
+            sum += off[e];
+            tsum += (off[e] + bm - 1) / bm;
+        }
+        int incl = sum, tincl = tsum;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int a = __shfl_up_sync(0xFFFFFFFFu, incl, d), b = __shfl_up_sync(0xFFFFFFFFu, tincl, d);
+            if (lane >= d) {
+                incl += a;
+                tincl += b;
+            }
+        }
+        int run = incl - sum, trun = tincl - tsum;
+        for (int e = e0; e < e1; ++e) {
             const int c = off[e];
             counts[e] = c;
             offsets[e] = run;
@@ -89,11 +137,14 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
             run += c;
             trun += (c + bm - 1) / bm;
         }
-        offsets[E] = run;
-        tile_offsets[E] = trun;
-        off[E] = run;
+        if (lane == 31) {
+            offsets[E] = incl;
+            tile_offsets[E] = tincl;
+            off[E] = incl;
+        }
     }
     __syncthreads();
+    int32_t *const place = staged ? sorted_s : sorted_pairs;
     for (int64_t base = beg; base < end; base += 32) {
         const int64_t p = base + lane;
         const int e = (p < end) ? expert_of(p) : -1;
@@ -104,11 +155,19 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
         const int wbase = valid ? cnt[warp * E + e] : 0;
         __syncwarp();
         if (valid && in_bounds(off[e] + wbase + rank, P)) {
-            sorted_pairs[off[e] + wbase + rank] = (int32_t)p;
+            place[off[e] + wbase + rank] = (int32_t)p;
             if (rank == 0) cnt[warp * E + e] = wbase + __popc(peers);
         }
         if (pair_rows && p < end) pair_rows[p] = valid ? off[e] + wbase + rank : -1;
         __syncwarp();
+    }
+    if (staged) {
+        __syncthreads();
+        const int rows = off[E];
+        const int nv = ((reinterpret_cast<uintptr_t>(sorted_pairs) & 15u) == 0) ? rows / 4 : 0;
+        for (int i = threadIdx.x; i < nv; i += blockDim.x)
+            reinterpret_cast<int4 *>(sorted_pairs)[i] = reinterpret_cast<const int4 *>(sorted_s)[i];
+        for (int i = 4 * nv + threadIdx.x; i < rows; i += blockDim.x) sorted_pairs[i] = sorted_s[i];
     }
 }
 
