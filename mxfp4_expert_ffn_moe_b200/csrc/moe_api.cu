@@ -474,18 +474,24 @@ int config_tok(TileConfig c) {
     }
 }
 
-// Pair permutation (one CTA).  The ids and the placed pairs are staged in shared
-// memory when they fit (up to ~35K pairs).
+// Pair permutation: about one CTA per 2048 pairs (at most 64 unless the sub-chunk
+// ids would not fit in shared memory), each placing its own range.
 int launch_permute(const int32_t *ids, int expert_base, int64_t P, int64_t E, int tile_rows, int32_t *counts,
                    int32_t *offsets, int32_t *tile_offsets, int32_t *sorted_pairs, int32_t *pair_rows,
                    cudaStream_t s) {
     const size_t cap = std::min<size_t>(moe::kPermuteSmemCap, (size_t)max_smem_optin());
-    const bool perm_attr = ensure_smem_attr(reinterpret_cast<const void *>(moe::permute_pairs_kernel), (int)cap);
-    const bool staged = perm_attr && moe::permute_smem_bytes((int)E, P, true) <= cap;
-    const size_t perm_smem = moe::permute_smem_bytes((int)E, P, staged);
+    const size_t fixed = moe::permute_smem_bytes((int)E, 0);
+    if (fixed + 64 > cap) return MOE_ERR_UNSUPPORTED;
+    const int64_t sc_max = (int64_t)((cap - fixed) / 64);
+    int64_t C = std::min<int64_t>(std::max<int64_t>(1, moe::ceil_div(P, moe::kPermutePairsPerCta)), 64);
+    if (moe::permute_subchunk(P, (int)C) > sc_max) C = moe::ceil_div(P, 32 * sc_max);
+    if (C > 0x7FFFFFFF) return MOE_ERR_INVALID_ARG;
+    const size_t smem = moe::permute_smem_bytes((int)E, moe::permute_subchunk(P, (int)C));
+    if (!ensure_smem_attr(reinterpret_cast<const void *>(moe::permute_pairs_kernel), (int)smem))
+        return MOE_ERR_CUDA;
     StageScope sp(MOE_STAGE_PERMUTE, s);
-    launch_pdl(moe::permute_pairs_kernel, dim3(1), dim3(moe::kPermuteThreads), perm_smem, s, ids, expert_base, P,
-               (int)E, tile_rows, staged ? 1 : 0, counts, offsets, tile_offsets, sorted_pairs, pair_rows);
+    launch_pdl(moe::permute_pairs_kernel, dim3((unsigned)C), dim3(moe::kPermuteThreads), smem, s, ids, expert_base,
+               P, (int)E, tile_rows, counts, offsets, tile_offsets, sorted_pairs, pair_rows);
     return launch_check();
 }
 

@@ -11,30 +11,31 @@
 //   pair_rows[p]     (optional) the inverse: the row of pair p, -1 for a dropped pair
 // Ids outside [0, E) raise MOE_DEVERR_BAD_EXPERT_ID and their pairs are dropped.
 //
-// One CTA of 32 warps: warp w owns a contiguous chunk of pairs, counts its experts
-// in a private shared-memory row, the chunk bases come from an exclusive scan over
-// warps (the expert starts from one warp's shuffle scan), and each warp then places
-// its chunk in order using __match_any_sync to rank equal experts inside a 32-pair
-// step.  When they fit (staged != 0, up to ~35K pairs), the ids are first copied
-// into shared memory as 16-bit expert numbers with coalesced 16-byte loads, the pairs
-// are placed into a shared-memory copy of sorted_pairs, and that copy leaves with
-// coalesced 16-byte stores: one SM alone would otherwise issue one L2 transaction per
-// pair for the scattered stores.
+// C CTAs of 32 warps, with no communication between them.  The pairs are cut into
+// 32*C sub-chunks of sc consecutive pairs; CTA c places the 32 sub-chunks of its range
+// [c*32*sc, (c+1)*32*sc), warp w the w-th of them.  Every CTA reads all the ids and
+// counts, per expert, the pairs before its range, in each of its sub-chunks and after
+// its range (warp-private rows, so shared atomics only collide inside a warp); from
+// these it has the totals (CTA 0 writes counts, offsets and tile_offsets), the expert
+// starts (one warp's shuffle scan) and the first row of each of its sub-chunks in each
+// expert.  Each warp then places its sub-chunk 32 pairs at a time, ranking equal
+// experts with __match_any_sync.  The ranking is the costly step (match.any issues at
+// about one per 32 clocks on an SM), which is why the pairs are spread over ~P/2048
+// CTAs instead of one.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int kPermuteThreads = 1024;
+constexpr int kPermutePairsPerCta = 2048;
 
-// Dynamic shared memory of permute_pairs_kernel: the count rows and expert starts;
-// when staged, also the P ids (int16) and the P placed pairs (int32, 16-byte aligned).
-__host__ __device__ constexpr size_t permute_ids_offset(int E) { return sizeof(int) * (size_t)(33 * E + 1); }
-__host__ __device__ constexpr size_t permute_sorted_offset(int E, int64_t P) {
-    return (permute_ids_offset(E) + 2 * (size_t)P + 15) & ~(size_t)15;
-}
-__host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t P, bool staged) {
-    return staged ? permute_sorted_offset(E, P) + 4 * (size_t)P : permute_ids_offset(E);
+// Sub-chunk length for C CTAs.
+__host__ __device__ constexpr int64_t permute_subchunk(int64_t P, int C) { return (P + 32 * (int64_t)C - 1) / (32 * (int64_t)C); }
+// Dynamic shared memory of permute_pairs_kernel: three [32][E] count tables, the E + 1
+// expert starts, and the CTA's sub-chunk ids (int16).
+__host__ __device__ constexpr size_t permute_smem_bytes(int E, int64_t sc) {
+    return sizeof(int) * (size_t)(3 * 32 * E + E + 1) + 2 * (size_t)(32 * sc);
 }
 constexpr size_t kPermuteSmemCap = 227 * 1024;
 
@@ -47,65 +48,73 @@ __device__ __forceinline__ int relative_expert(int32_t id, int expert_base, int 
 // of the E experts handled here (a rank's slice of the experts under expert parallelism;
 // 0 for the whole layer).
 __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
-    const int32_t *__restrict__ ids, int expert_base, int64_t P, int E, int bm, int staged, int32_t *__restrict__ counts,
+    const int32_t *__restrict__ ids, int expert_base, int64_t P, int E, int bm, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tile_offsets,
     int32_t *__restrict__ sorted_pairs, int32_t *__restrict__ pair_rows) {
     pdl_wait();
     pdl_trigger();
-    extern __shared__ __align__(16) unsigned char sm_perm_raw[];
-    int *cnt = reinterpret_cast<int *>(sm_perm_raw);     // [32][E]: per-warp counts, then running bases
-    int *off = cnt + 32 * E;                              // [E + 1]: expert start rows
-    int16_t *ids_s = reinterpret_cast<int16_t *>(sm_perm_raw + permute_ids_offset(E));          // [P]
-    int32_t *sorted_s = reinterpret_cast<int32_t *>(sm_perm_raw + permute_sorted_offset(E, P));  // [P]
+    extern __shared__ __align__(16) int sm_perm[];
+    int *pre = sm_perm;                 // [32][E]: per-warp counts before the range
+    int *post = pre + 32 * E;           // [32][E]: per-warp counts after the range
+    int *cnt = post + 32 * E;           // [32][E]: per-sub-chunk counts, then first rows
+    int *off = cnt + 32 * E;            // [E + 1]: expert start rows
+    int16_t *ids_s = reinterpret_cast<int16_t *>(off + E + 1);   // [32 * sc]: the range's experts
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) cnt[i] = 0;
-    if (staged) {
-        // 16-byte loads, eight per thread in flight before their stores
-        const int64_t nv = ((reinterpret_cast<uintptr_t>(ids) & 15u) == 0) ? P / 4 : 0;
-        const int4 *ids4 = reinterpret_cast<const int4 *>(ids);
-        for (int64_t i0 = threadIdx.x; i0 < nv; i0 += 8 * (int64_t)blockDim.x) {
-            int4 v[8];
+    const int64_t sc = permute_subchunk(P, gridDim.x);
+    const int64_t own_beg = min(P, (int64_t)blockIdx.x * 32 * sc);
+    const int64_t own_end = min(P, own_beg + 32 * sc);
+    // one CTA: every pair is in its range, the before/after tables stay unused
+    const bool single = gridDim.x == 1;
+    for (int i = threadIdx.x + (single ? 2 * 32 * E : 0); i < 3 * 32 * E; i += blockDim.x) sm_perm[i] = 0;
+    __syncthreads();
+
+    auto count_pair = [&](int64_t i, int32_t id) {
+        const int e = relative_expert(id, expert_base, E);
+        if (i < own_beg) {
+            if (e >= 0) atomicAdd(&pre[warp * E + e], 1);
+        } else if (i < own_end) {
+            ids_s[i - own_beg] = (int16_t)e;
+            if (e >= 0)
+                atomicAdd(&cnt[(int)((i - own_beg) / sc) * E + e], 1);
+            else
+                raise_device_error(MOE_DEVERR_BAD_EXPERT_ID);
+        } else if (e >= 0) {
+            atomicAdd(&post[warp * E + e], 1);
+        }
+    };
+    // all ids: 16-byte loads, four per thread in flight before their counts
+    const int64_t nv = ((reinterpret_cast<uintptr_t>(ids) & 15u) == 0) ? P / 4 : 0;
+    const int4 *ids4 = reinterpret_cast<const int4 *>(ids);
+    for (int64_t i0 = threadIdx.x; i0 < nv; i0 += 4 * (int64_t)blockDim.x) {
+        int4 v[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (i0 + u * (int64_t)blockDim.x < nv) v[u] = __ldg(ids4 + i0 + u * (int64_t)blockDim.x);
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * (int64_t)blockDim.x < nv) v[u] = __ldg(ids4 + i0 + u * (int64_t)blockDim.x);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int64_t i = i0 + u * (int64_t)blockDim.x;
-                if (i >= nv) continue;
-                ids_s[4 * i] = (int16_t)relative_expert(v[u].x, expert_base, E);
-                ids_s[4 * i + 1] = (int16_t)relative_expert(v[u].y, expert_base, E);
-                ids_s[4 * i + 2] = (int16_t)relative_expert(v[u].z, expert_base, E);
-                ids_s[4 * i + 3] = (int16_t)relative_expert(v[u].w, expert_base, E);
+        for (int u = 0; u < 4; ++u) {
+            const int64_t i = i0 + u * (int64_t)blockDim.x;
+            if (i >= nv) continue;
+            count_pair(4 * i, v[u].x);
+            count_pair(4 * i + 1, v[u].y);
+            count_pair(4 * i + 2, v[u].z);
+            count_pair(4 * i + 3, v[u].w);
+        }
+    }
+    for (int64_t i = 4 * nv + threadIdx.x; i < P; i += blockDim.x) count_pair(i, __ldg(ids + i));
+    __syncthreads();
+    // per expert: the totals, then (after the scan) the first row of each sub-chunk
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int before = 0, total = 0;
+        if (single) {
+            for (int w = 0; w < 32; ++w) total += cnt[w * E + e];
+        } else {
+            for (int w = 0; w < 32; ++w) {
+                before += pre[w * E + e];
+                total += cnt[w * E + e] + post[w * E + e];
             }
         }
-        for (int64_t i = 4 * nv + threadIdx.x; i < P; i += blockDim.x)
-            ids_s[i] = (int16_t)relative_expert(__ldg(ids + i), expert_base, E);
-    }
-    __syncthreads();
-    // expert of pair p relative to expert_base, -1 when outside [0, E)
-    auto expert_of = [&](int64_t p) {
-        return staged ? (int)ids_s[p] : relative_expert(__ldg(ids + p), expert_base, E);
-    };
-
-    const int64_t chunk = (P + 31) / 32;
-    const int64_t beg = (int64_t)warp * chunk;
-    const int64_t end = (beg + chunk < P) ? beg + chunk : P;
-    for (int64_t p = beg + lane; p < end; p += 32) {
-        const int e = expert_of(p);
-        if ((unsigned)e < (unsigned)E)
-            atomicAdd(&cnt[warp * E + e], 1);
-        else
-            raise_device_error(MOE_DEVERR_BAD_EXPERT_ID);
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int w = 0; w < 32; ++w) {
-            const int c = cnt[w * E + e];
-            cnt[w * E + e] = run;
-            run += c;
-        }
-        off[e] = run;
+        off[e] = before + total;
+        pre[e] = before;              // row 0 of pre is only read again as the "before" count
     }
     __syncthreads();
     if (warp == 0) {
@@ -130,44 +139,50 @@ __global__ void __launch_bounds__(kPermuteThreads) permute_pairs_kernel(
         int run = incl - sum, trun = tincl - tsum;
         for (int e = e0; e < e1; ++e) {
             const int c = off[e];
-            counts[e] = c;
-            offsets[e] = run;
-            tile_offsets[e] = trun;
+            if (blockIdx.x == 0) {
+                counts[e] = c;
+                offsets[e] = run;
+                tile_offsets[e] = trun;
+            }
             off[e] = run;
             run += c;
             trun += (c + bm - 1) / bm;
         }
         if (lane == 31) {
-            offsets[E] = incl;
-            tile_offsets[E] = tincl;
+            if (blockIdx.x == 0) {
+                offsets[E] = incl;
+                tile_offsets[E] = tincl;
+            }
             off[E] = incl;
         }
     }
     __syncthreads();
-    int32_t *const place = staged ? sorted_s : sorted_pairs;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = off[e] + pre[e];
+        for (int w = 0; w < 32; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const int64_t beg = min(own_end, own_beg + warp * sc);
+    const int64_t end = min(own_end, beg + sc);
     for (int64_t base = beg; base < end; base += 32) {
         const int64_t p = base + lane;
-        const int e = (p < end) ? expert_of(p) : -1;
-        const bool valid = (p < end) && (unsigned)e < (unsigned)E;
+        const int e = (p < end) ? (int)ids_s[p - own_beg] : -1;
+        const bool valid = (p < end) && e >= 0;
         const int key = valid ? e : -1 - lane;
         const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
         const int rank = __popc(peers & ((1u << lane) - 1u));
-        const int wbase = valid ? cnt[warp * E + e] : 0;
+        const int row = valid ? cnt[warp * E + e] + rank : -1;
         __syncwarp();
-        if (valid && in_bounds(off[e] + wbase + rank, P)) {
-            place[off[e] + wbase + rank] = (int32_t)p;
-            if (rank == 0) cnt[warp * E + e] = wbase + __popc(peers);
+        if (valid && in_bounds(row, P)) {
+            sorted_pairs[row] = (int32_t)p;
+            if (rank == 0) cnt[warp * E + e] += __popc(peers);
         }
-        if (pair_rows && p < end) pair_rows[p] = valid ? off[e] + wbase + rank : -1;
+        if (pair_rows && p < end) pair_rows[p] = row;
         __syncwarp();
-    }
-    if (staged) {
-        __syncthreads();
-        const int rows = off[E];
-        const int nv = ((reinterpret_cast<uintptr_t>(sorted_pairs) & 15u) == 0) ? rows / 4 : 0;
-        for (int i = threadIdx.x; i < nv; i += blockDim.x)
-            reinterpret_cast<int4 *>(sorted_pairs)[i] = reinterpret_cast<const int4 *>(sorted_s)[i];
-        for (int i = 4 * nv + threadIdx.x; i < rows; i += blockDim.x) sorted_pairs[i] = sorted_s[i];
     }
 }
 
