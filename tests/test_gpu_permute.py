@@ -59,7 +59,8 @@ def _check(moe, ids_np, E, tile_rows):
     (37, 3, 7, 32),         # ragged tails
     (4096, 4, 32, 256),     # the gpt-oss-20b prefill layer's shape
     (2048, 8, 256, 32),     # largest E and k
-    (15000, 4, 64, 256),    # 60,000 pairs: past the shared-memory staging of the ids
+    (15000, 4, 64, 256),    # 60,000 pairs: 30 CTAs, each placing its own range
+    (40000, 4, 128, 256),   # 160,000 pairs: the 64-CTA cap, sub-chunks of 79 pairs
 ])
 def test_permute_uniform_ids(moe_gpu, T, k, E, tile_rows):
     rng = np.random.default_rng(T * 7 + E)
